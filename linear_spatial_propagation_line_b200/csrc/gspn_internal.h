@@ -1,0 +1,42 @@
+// Internal launch interface between the C ABI (gspn_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gspn_common.cuh"
+
+namespace gspn {
+
+// One validated call: directions [d0, d1) of the four-direction operation.
+// For a single-direction call the pointer arrays hold the tensors at index d0.
+struct Problem {
+    const void* x;
+    Ptr4 z;    // wlogit[d]: [B][C][3][H][W]
+    Ptr4 lam;  // [B][C][H][W]
+    Ptr4 u;    // [B][C][H][W]
+    int64_t B, C, H, W, g;
+    int dtype;  // GSPN_F32 / GSPN_BF16
+    int d0, d1;
+    cudaStream_t stream;
+    void* y;
+    cudaEvent_t ev_begin = nullptr;  // recorded around the dominant kernel if set
+    cudaEvent_t ev_end = nullptr;
+    const char* kernel_name = "";   // set by the launcher: the dominant kernel
+    int64_t planes() const { return B * C; }
+    int64_t pixch() const { return B * C * H * W; }
+};
+
+// Whole-plane kernel: one CTA keeps a plane's fp32 output and one direction's
+// weights in shared memory.  Used when max(H, W) <= 64 and the plane fits.
+bool small_plane_fits(const Problem& pb, size_t* smem_bytes);
+cudaError_t launch_small_plane(Problem& pb, int* launches);
+
+// Generic line-chain path for any plane size: one CTA per (plane, direction)
+// scans with the whole line in shared memory and adds u_d * h_d into the fp32
+// workspace `ws` (B*C*H*W floats, zeroed here), then a conversion kernel
+// writes y.
+cudaError_t launch_chain(Problem& pb, float* ws, int* launches);
+
+}  // namespace gspn

@@ -1,0 +1,203 @@
+"""Python binding of the GSPN C ABI (``include/gspn.h``).
+
+Argument marshalling only: tensors are checked and turned into raw pointers,
+and every step of the propagation runs in the CUDA library
+``_lib/libgspn_b200.so``.  There is no CPU or PyTorch fallback: if the
+library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+import torch
+
+from . import build as _build
+
+GSPN_F32 = 0
+GSPN_BF16 = 1
+_DTYPES = {torch.float32: GSPN_F32, torch.bfloat16: GSPN_BF16}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class GSPNError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"gspn status {status}: {message}")
+        self.status = status
+
+
+def library_path():
+    return _build.LIB_PATH
+
+
+def load_library():
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = _build.LIB_PATH
+        if not path.exists():
+            raise RuntimeError(
+                f"GSPN CUDA library not found at {path}; build it with "
+                "`python -m linear_spatial_propagation_line_b200.build`")
+        lib = ctypes.CDLL(str(path))
+        vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        arr4 = vp * 4
+        lib.gspn_forward.argtypes = [vp, arr4, arr4, arr4, i64, i64, i64, i64, i64, ci, vp, vp]
+        lib.gspn_forward.restype = ci
+        lib.gspn_forward_dir.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, ci, ci, vp, vp]
+        lib.gspn_forward_dir.restype = ci
+        lib.gspn_forward_host.argtypes = [vp, arr4, arr4, arr4, i64, i64, i64, i64, i64, ci, vp,
+                                          vp]
+        lib.gspn_forward_host.restype = ci
+        for name in ("gspn_last_launch_count", "gspn_release", "gspn_version"):
+            getattr(lib, name).argtypes = []
+            getattr(lib, name).restype = ci
+        lib.gspn_status_string.argtypes = [ci]
+        lib.gspn_status_string.restype = ctypes.c_char_p
+        lib.gspn_last_cuda_error.argtypes = []
+        lib.gspn_last_cuda_error.restype = ctypes.c_char_p
+        lib.gspn_set_timing_events.argtypes = [vp, vp]
+        lib.gspn_set_timing_events.restype = ci
+        lib.gspn_last_kernel_name.argtypes = []
+        lib.gspn_last_kernel_name.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def _check(status: int):
+    if status != 0:
+        lib = load_library()
+        msg = lib.gspn_status_string(status).decode()
+        if status == -6:
+            msg += ": " + lib.gspn_last_cuda_error().decode()
+        raise GSPNError(status, msg)
+
+
+def status_string(status: int) -> str:
+    return load_library().gspn_status_string(status).decode()
+
+
+def version() -> int:
+    return load_library().gspn_version()
+
+
+def last_launch_count() -> int:
+    """Kernels launched by this thread's most recent successful forward call."""
+    return load_library().gspn_last_launch_count()
+
+
+def set_timing_events(begin=None, end=None):
+    """Record torch.cuda.Event ``begin``/``end`` around the dominant kernel of
+    every later forward call on this thread (None, None stops)."""
+    b = ctypes.c_void_p(begin.cuda_event) if begin is not None else None
+    e = ctypes.c_void_p(end.cuda_event) if end is not None else None
+    _check(load_library().gspn_set_timing_events(b, e))
+
+
+def last_kernel_name() -> str:
+    return load_library().gspn_last_kernel_name().decode()
+
+
+def release():
+    """Free the current device's workspace and staging buffers."""
+    _check(load_library().gspn_release())
+
+
+def _shape_of(x):
+    if x.dim() != 4:
+        raise ValueError("x must be [B,C,H,W]")
+    return tuple(int(s) for s in x.shape)
+
+
+def _validate(x, wlogit, lam, u, dirs, device_kind):
+    B, C, H, W = _shape_of(x)
+    if x.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {x.dtype}")
+    tensors = [x]
+    for d in dirs:
+        if tuple(wlogit[d].shape) != (B, C, 3, H, W):
+            raise ValueError(f"wlogit[{d}] must be [B,C,3,H,W], got {tuple(wlogit[d].shape)}")
+        for name, t in (("lam", lam[d]), ("u", u[d])):
+            if tuple(t.shape) != (B, C, H, W):
+                raise ValueError(f"{name}[{d}] must be [B,C,H,W], got {tuple(t.shape)}")
+        tensors += [wlogit[d], lam[d], u[d]]
+    for t in tensors:
+        if t.dtype != x.dtype:
+            raise TypeError("every tensor must have x's dtype")
+        if not t.is_contiguous():
+            raise ValueError("every tensor must be contiguous")
+        if device_kind == "cuda" and (not t.is_cuda or t.device != x.device):
+            raise ValueError("every tensor must be on x's CUDA device")
+        if device_kind == "cpu" and t.is_cuda:
+            raise ValueError("forward_host takes host tensors")
+    return B, C, H, W
+
+
+def _stream_handle(device, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def forward(x, wlogit, lam, u, group_len: int = 0, out=None, stream=None):
+    """y = sum_d u[d] * h_d on CUDA tensors (see include/gspn.h)."""
+    lib = load_library()
+    B, C, H, W = _validate(x, wlogit, lam, u, range(4), "cuda")
+    y = torch.empty_like(x) if out is None else out
+    _validate(y, wlogit, lam, u, [], "cuda")
+    arr4 = ctypes.c_void_p * 4
+    with torch.cuda.device(x.device):
+        st = _stream_handle(x.device, stream)
+        _check(lib.gspn_forward(x.data_ptr(), arr4(*[t.data_ptr() for t in wlogit]),
+                                arr4(*[t.data_ptr() for t in lam]),
+                                arr4(*[t.data_ptr() for t in u]), B, C, H, W, int(group_len),
+                                _DTYPES[x.dtype], st, y.data_ptr()))
+    return y
+
+
+def forward_dir(x, wlogit_d, lam_d, u_d, d: int, group_len: int = 0, out=None, stream=None):
+    """y = u_d * h_d for one direction d on CUDA tensors."""
+    lib = load_library()
+    z = [wlogit_d] * 4
+    la = [lam_d] * 4
+    uu = [u_d] * 4
+    B, C, H, W = _validate(x, z, la, uu, [0], "cuda")
+    y = torch.empty_like(x) if out is None else out
+    with torch.cuda.device(x.device):
+        st = _stream_handle(x.device, stream)
+        _check(lib.gspn_forward_dir(x.data_ptr(), wlogit_d.data_ptr(), lam_d.data_ptr(),
+                                    u_d.data_ptr(), B, C, H, W, int(group_len), int(d),
+                                    _DTYPES[x.dtype], st, y.data_ptr()))
+    return y
+
+
+def forward_host(x, wlogit, lam, u, group_len: int = 0, out=None, device=None, stream=None):
+    """gspn_forward_host on CPU tensors (pinned memory makes the copies
+    asynchronous); returns y on the host, ready when the call returns."""
+    lib = load_library()
+    B, C, H, W = _validate(x, wlogit, lam, u, range(4), "cpu")
+    y = torch.empty_like(x) if out is None else out
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    arr4 = ctypes.c_void_p * 4
+    with torch.cuda.device(device):
+        st = _stream_handle(device, stream)
+        _check(lib.gspn_forward_host(x.data_ptr(), arr4(*[t.data_ptr() for t in wlogit]),
+                                     arr4(*[t.data_ptr() for t in lam]),
+                                     arr4(*[t.data_ptr() for t in u]), B, C, H, W,
+                                     int(group_len), _DTYPES[x.dtype], st, y.data_ptr()))
+    return y
+
+
+def raw_forward(ptrs: dict, shape, group_len: int, dtype: int, stream_handle: int) -> int:
+    """Direct C-ABI call on raw device pointers (for callers that manage their
+    own buffers); returns the status code without raising."""
+    lib = load_library()
+    arr4 = ctypes.c_void_p * 4
+    B, C, H, W = shape
+    return lib.gspn_forward(ptrs["x"], arr4(*ptrs["wlogit"]), arr4(*ptrs["lam"]),
+                            arr4(*ptrs["u"]), B, C, H, W, int(group_len), int(dtype),
+                            ctypes.c_void_p(stream_handle), ptrs["y"])
