@@ -145,7 +145,7 @@ class ClockSampler:
         self.path = None
         try:
             props = torch.cuda.get_device_properties(device_index)
-            self.bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}"
+            self.bus = f"{props.pci_bus_id:02X}:{props.pci_device_id:02X}."
         except Exception:
             self.bus = None
 
@@ -174,7 +174,7 @@ class ClockSampler:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
-            if self.bus and not parts[0].upper().endswith(self.bus[-7:]):
+            if self.bus and self.bus not in parts[0].upper():
                 continue
             rows.append(parts)
         try:
