@@ -46,6 +46,7 @@ L2_BYTES = 126 * 1024 * 1024
 KERNELS = {
     "small_plane_kernel": (["gspn_small.cu", "gspn_common.cuh"], 22),
     "chain_kernel": (["gspn_chain.cu", "gspn_common.cuh"], 21),
+    "fused_kernel": (["gspn_fused.cu", "gspn_ptx.cuh", "gspn_common.cuh"], 22),
 }
 CSRC = ROOT / "linear_spatial_propagation_line_b200" / "csrc"
 
@@ -57,6 +58,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--C", type=int, default=None,
+                    help="override the channel count (small cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -394,6 +397,8 @@ def measure_e2e(args, wl, inp, device, world):
 def main():
     args = parse_args()
     wl = WORKLOADS[args.workload]
+    if args.C is not None:
+        wl = wl.with_(C=args.C)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

@@ -122,6 +122,25 @@ int gspn_set_timing_events(void* begin, void* end);
  * thread (static storage; "" before the first call). */
 const char* gspn_last_kernel_name(void);
 
+/*
+ * Synchronises `stream` and reports whether a kernel of this library on the
+ * current device gave up a bounded device-side wait (a TMA stage, a halo
+ * exchange or a slot hand-over that did not arrive within its time limit).
+ * Returns GSPN_OK, or GSPN_ERR_TIMEOUT once per such event (the word is then
+ * cleared).  After such an event the large-plane kernel refuses further work
+ * (its calls leave y unwritten) until this function has been called; the
+ * next call after it starts from a cleared workspace.
+ */
+int gspn_check_device_status(void* stream);
+
+/*
+ * Test hook: the next large-plane launch on this thread waits for a slot
+ * hand-over that never happens, gives up after `timeout_ns` nanoseconds and
+ * records GSPN_ERR_TIMEOUT for gspn_check_device_status.  No GPU fault is
+ * involved.  Returns GSPN_OK, or GSPN_ERR_SHAPE if timeout_ns <= 0.
+ */
+int gspn_debug_force_timeout(int64_t timeout_ns);
+
 /* Frees the current device's workspace and staging area.  Not thread safe
  * against concurrent gspn_* calls on the same device. */
 int gspn_release(void);

@@ -16,8 +16,12 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 struct DeviceBuffers {
-    void* ws = nullptr;
+    void* ws = nullptr;  // fp32 accumulator of the line-chain path
     size_t ws_bytes = 0;
+    void* fused = nullptr;  // control block + L2 slots of the fused path (kept zeroed)
+    size_t fused_bytes = 0;
+    bool fused_dirty = false;    // slots may hold leftovers of an aborted launch
+    bool pending_error = false;  // a device error seen while replacing the workspace
     void* staging = nullptr;
     size_t staging_bytes = 0;
 };
@@ -30,6 +34,8 @@ thread_local int t_last_launches = 0;
 thread_local cudaEvent_t t_ev_begin = nullptr;
 thread_local cudaEvent_t t_ev_end = nullptr;
 thread_local const char* t_last_kernel = "";
+thread_local bool t_force_timeout = false;
+thread_local unsigned long long t_force_timeout_ns = 0;
 
 int cuda_fail(cudaError_t e) {
     snprintf(t_cuda_error, sizeof(t_cuda_error), "%s: %s", cudaGetErrorName(e),
@@ -130,13 +136,57 @@ int validate(const void* x, const void* const* wlogit, const void* const* lam,
     return GSPN_OK;
 }
 
+// The fused workspace: grown on demand, zero-filled when (re)allocated.
+int ensure_fused(DeviceBuffers& db, size_t need, cudaStream_t stream) {
+    if (db.fused_bytes >= need) return GSPN_OK;
+    if (db.fused) {
+        int sticky = 0;
+        cudaError_t e = cudaMemcpy(&sticky, static_cast<char*>(db.fused) +
+                                                gspn::kFusedStickyErrorOffset,
+                                   sizeof(int), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (sticky) db.pending_error = true;
+        e = cudaFree(db.fused);
+        db.fused = nullptr;
+        db.fused_bytes = 0;
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    cudaError_t e = cudaMalloc(&db.fused, need);
+    if (e != cudaSuccess) {
+        db.fused = nullptr;
+        return cuda_fail(e);
+    }
+    db.fused_bytes = need;
+    e = cudaMemsetAsync(db.fused, 0, need, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    db.fused_dirty = false;
+    return GSPN_OK;
+}
+
 int run(gspn::Problem& pb) {
     int launches = 0;
     pb.ev_begin = t_ev_begin;
     pb.ev_end = t_ev_end;
     cudaError_t e;
+    gspn::FusedPlan fp;
     if (gspn::small_plane_fits(pb, nullptr)) {
         e = gspn::launch_small_plane(pb, &launches);
+    } else if (gspn::fused_plan(pb, &fp)) {
+        int dev;
+        int s = current_device(&dev);
+        if (s != GSPN_OK) return s;
+        std::lock_guard<std::mutex> lock(g_mutex);
+        DeviceBuffers& db = g_dev[dev];
+        s = ensure_fused(db, fp.ws_bytes, pb.stream);
+        if (s != GSPN_OK) return s;
+        fp.zero_slots = db.fused_dirty;
+        db.fused_dirty = false;
+        if (t_force_timeout) {
+            fp.force_stale = 1;
+            fp.timeout_ns = t_force_timeout_ns;
+            t_force_timeout = false;
+        }
+        e = gspn::launch_fused(pb, fp, db.fused, &launches);
     } else {
         int dev;
         int s = current_device(&dev);
@@ -233,6 +283,41 @@ int gspn_forward_host(const void* x, const void* const wlogit[4], const void* co
 
 int gspn_last_launch_count(void) { return t_last_launches; }
 
+int gspn_check_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    int dev;
+    int s = current_device(&dev);
+    if (s != GSPN_OK) return s;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceBuffers& db = g_dev[dev];
+    bool failed = db.pending_error;
+    db.pending_error = false;
+    if (db.fused) {
+        int sticky = 0;
+        char* word = static_cast<char*>(db.fused) + gspn::kFusedStickyErrorOffset;
+        e = cudaMemcpy(&sticky, word, sizeof(int), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (sticky) {
+            e = cudaMemset(word, 0, sizeof(int));
+            if (e != cudaSuccess) return cuda_fail(e);
+            failed = true;
+        }
+    }
+    if (failed) {
+        db.fused_dirty = true;
+        return GSPN_ERR_TIMEOUT;
+    }
+    return GSPN_OK;
+}
+
+int gspn_debug_force_timeout(int64_t timeout_ns) {
+    if (timeout_ns <= 0) return GSPN_ERR_SHAPE;
+    t_force_timeout = true;
+    t_force_timeout_ns = (unsigned long long)timeout_ns;
+    return GSPN_OK;
+}
+
 int gspn_set_timing_events(void* begin, void* end) {
     t_ev_begin = static_cast<cudaEvent_t>(begin);
     t_ev_end = static_cast<cudaEvent_t>(end);
@@ -249,6 +334,10 @@ int gspn_release(void) {
     DeviceBuffers& db = g_dev[dev];
     cudaError_t e = cudaSuccess;
     if (db.ws) e = cudaFree(db.ws);
+    if (db.fused) {
+        cudaError_t e2 = cudaFree(db.fused);
+        if (e == cudaSuccess) e = e2;
+    }
     if (db.staging) {
         cudaError_t e2 = cudaFree(db.staging);
         if (e == cudaSuccess) e = e2;

@@ -1,0 +1,1019 @@
+// Fused persistent GSPN kernel for large planes (sm_100a).
+//
+// What it computes: for every (b, c) plane and direction d, the line recurrence
+//   h_i = w_i h_{i-1} + lambda_i (.) x_i,   h = lambda (.) x on a group's first line
+// with three-neighbour row-stochastic weights (sigmoid, then normalisation over
+// the existing neighbours), and y = sum_d u_d (.) h_d -- CSDN walkthrough
+// "GSPN——在convolution基础上并行序列建模", sections "方法", "如何设计一个高效的
+// 传播层", "行随机矩阵" and "全局与局部GSPN".
+//
+// How (B200 design):
+//  * Work item = one (plane, direction) chain.  A team of S CTAs (one thread
+//    block cluster, one CTA per SM) runs a chain; CTA j owns positions
+//    [j*Kc, (j+1)*Kc) of the line and also recomputes a halo of kHalo positions
+//    on each side.  A halo value stays exact for kHalo steps after a refresh,
+//    so neighbouring CTAs exchange their edge states only every kHalo steps,
+//    through DSMEM `st.async` stores that complete transaction bytes on the
+//    receiver's mbarrier.
+//  * Each thread owns two adjacent positions and does the arithmetic on packed
+//    fp32 pairs (sm_100 f32x2 FMA/MUL/ADD), so every instruction but the
+//    exponentials and reciprocals serves two pixels.  The previous line lives
+//    in a double-buffered shared-memory line; one named barrier over the
+//    active warps per step.
+//  * Inputs stream through a kStages-deep shared-memory ring filled by TMA
+//    tensor loads (no multicast): vertical scans load R rows x (Kc + 2*kHalo)
+//    columns per stage; horizontal scans load (Kc + 2*kHalo) rows x 16 bytes,
+//    so each thread reads its two row segments with 16-byte shared loads and
+//    the scan runs along W with no transposition copy.
+//  * The four chains of a plane accumulate u_d * h_d into an fp32 "slot" kept
+//    L2-resident (evict_last reductions; streaming inputs use evict_first).
+//    The team that finishes a plane's last chain rounds the slot to the output
+//    dtype once, writes y, re-zeroes the slot and releases it.  A ring of
+//    n_slots slots bounds the L2 footprint; teams take items from a global
+//    queue in plane-major order, so every plane a team waits for has already
+//    been handed to running teams (no deadlock).
+//  * Every wait (TMA stage, halo, slot release) is bounded by a global-timer
+//    limit; on expiry the kernel records an error word and winds down.
+//
+// Weights: with a_o = 1 + exp(-z_o), w_o = prod_{o' != o} a_o' / sum_o prod_{o'
+// != o} a_o' over the existing neighbours (3 exponentials + 1 reciprocal per
+// pixel).  Every a_o is computed scaled by 2^-32, which cancels in the ratio and
+// keeps the products finite unless two neighbour logits of one pixel sum to
+// less than about -133.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <stdio.h>
+#include <stdlib.h>
+
+#include <type_traits>
+#include <utility>
+
+#include "gspn_internal.h"
+#include "gspn_ptx.cuh"
+
+namespace gspn {
+namespace {
+
+using ptx::f2;
+
+constexpr int kMaxStages = 3;
+constexpr int kMaxSlots = 64;
+constexpr int kHalo = 32;        // halo width == steps between exchanges
+constexpr int kMaxThreads = 640; // one position per consumer thread + one producer warp
+
+// Control block in global memory (the first bytes of the fused workspace).
+struct FusedCtrl {
+    int sticky_error;  // kept across calls until the host reads it
+    int pad0[3];
+    int call_error;    // this call: nonzero stops every team (1 TMA, 2 slot, 3 halo, 4 stale)
+    int next_item;
+    int pad1[10];
+    int slot_epoch[kMaxSlots];
+    // int plane_done[planes] follows
+};
+constexpr size_t kCtrlResetOffset = 16;  // bytes before this survive the per-call reset
+
+struct __align__(64) FusedParams {
+    CUtensorMap tm_xv;     // x with vertical boxes
+    CUtensorMap tm_xh;     // x with horizontal boxes
+    CUtensorMap tm_z[4];   // logits of direction d (boxes of d's orientation)
+    CUtensorMap tm_l[4];
+    CUtensorMap tm_u[4];
+    void* y;
+    float* slots;
+    FusedCtrl* ctrl;
+    int* plane_done;
+    unsigned long long timeout_ns;
+    int H, W, planes, g;
+    int d0, nd;            // directions [d0, d0 + nd)
+    int S;                 // team size (CTAs per cluster)
+    int Kc_v, Kc_h;        // owned positions per CTA (vertical / horizontal scans)
+    int np_v, np_h;        // positions handled per CTA (owned + halos)
+    int nb_v, bw_v, R_v;   // vertical: column boxes, box width, rows per stage
+    int box_v;             // bytes between vertical boxes in a tile (128-aligned)
+    int nb_h, bh_h;        // horizontal: row boxes, box height (multiple of 8)
+    int tile_bytes;        // one tensor's tile in one stage
+    int stages;            // depth of the shared-memory ring (2 or 3)
+    int J_h;               // horizontal steps per stage (32-byte row segments)
+    int n_slots;
+    int n_items;
+    int force_stale;       // test hook: expect a slot epoch that never comes
+};
+
+// Shared-memory carve-up (dynamic shared memory).
+struct SmemView {
+    char* ring;
+    float* hb;   // 2 lines of (np_max + 4) floats; position p at index p + 2
+    float* rx;   // [2 parity][2 side][kHalo]
+    uint64_t* full_bar;   // [stages] TMA completion (expect_tx by the producer warp)
+    uint64_t* empty_bar;  // [stages] slot released by the consumers (one arrival)
+    uint64_t* halo_bar;   // [2] halo data arrived from the neighbour CTAs
+    int* cell;   // [0] item, [1] convert decision, [2] full phases, [3] halo phases
+    int line;    // floats per line buffer
+    int tile_bytes;
+    __device__ char* tile(int stage, int tensor) const {
+        return ring + (size_t)(stage * 6 + tensor) * tile_bytes;
+    }
+};
+
+__host__ __device__ inline size_t smem_layout(int tile_bytes, int stages, int npmax,
+                                              size_t* off_hb, size_t* off_rx, size_t* off_bar) {
+    size_t off = (size_t)stages * 6 * tile_bytes;
+    *off_hb = off;
+    off += sizeof(float) * 2 * (size_t)(npmax + 4);
+    *off_rx = off;
+    off += sizeof(float) * 2 * 2 * kHalo;
+    off = (off + 7) & ~(size_t)7;
+    *off_bar = off;
+    off += sizeof(uint64_t) * (2 * kMaxStages + 2) + 4 * sizeof(int);
+    return off;
+}
+
+__device__ __forceinline__ SmemView carve(char* base, const FusedParams& p) {
+    const int npmax = p.np_v > p.np_h ? p.np_v : p.np_h;
+    size_t ohb, orx, obar;
+    smem_layout(p.tile_bytes, p.stages, npmax, &ohb, &orx, &obar);
+    SmemView v;
+    v.tile_bytes = p.tile_bytes;
+    v.ring = base;
+    v.line = npmax + 4;
+    v.hb = reinterpret_cast<float*>(base + ohb);
+    v.rx = reinterpret_cast<float*>(base + orx);
+    v.full_bar = reinterpret_cast<uint64_t*>(base + obar);
+    v.empty_bar = v.full_bar + kMaxStages;
+    v.halo_bar = v.empty_bar + kMaxStages;
+    v.cell = reinterpret_cast<int*>(v.halo_bar + 2);
+    return v;
+}
+
+// Calls f(std::integral_constant<int, I>{}) for I = 0..N-1 (compile-time indices).
+template <class F, int... Is>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>) {
+    (f(std::integral_constant<int, Is>{}), ...);
+}
+template <int N, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+    static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+// Per-thread view of the mbarrier phases (identical in every active thread;
+// thread 0 publishes them in shared memory between chains).
+struct Phases {
+    uint32_t full;  // bit s: parity to wait for on full_bar[s]
+    uint32_t halo;  // bit p: parity to wait for on halo_bar[p]
+    bool abort;     // a bounded wait expired: skip further waits
+};
+
+__device__ __forceinline__ void report_error(const FusedParams& p, int code) {
+    atomicCAS(&p.ctrl->call_error, 0, code);
+    atomicCAS(&p.ctrl->sticky_error, 0, code);
+}
+
+__device__ __forceinline__ void wait_bar(const FusedParams& p, Phases& ph, uint64_t* bar,
+                                         uint32_t parity, int code) {
+    if (ph.abort) return;
+    if (!ptx::wait_parity_bounded(ptx::smem_addr(bar), parity, p.timeout_ns)) {
+        ph.abort = true;
+        report_error(p, code);
+    }
+}
+
+// Element e of a 16-byte vector of bf16 (e < 8) or fp32 (e < 4); e folds to a
+// constant inside fully unrolled loops.
+template <class T>
+__device__ __forceinline__ float vec_elem(const uint4& v, int e) {
+    if constexpr (sizeof(T) == 4) {
+        return __uint_as_float(e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w);
+    } else {
+        const int q = e >> 1;
+        const uint32_t w = q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+        return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+    }
+}
+
+// Thread 0 arms halo barrier (blk & 1) for block blk if that block ends in an
+// exchange (block blk covers steps [blk*kHalo, (blk+1)*kHalo) and exchanges
+// after its last step when more steps follow).  Blocks 0 and 1 are armed at
+// chain start; block b+2 right after block b's exchange completed on this CTA,
+// which is before any neighbour can send block b+2's data.
+__device__ __forceinline__ void arm_halo_block(const FusedParams& p, const SmemView& sm, int rank,
+                                               int blk, int L) {
+    if ((blk + 1) * kHalo < L) {
+        const uint32_t bytes =
+            sizeof(float) * kHalo * ((rank > 0 ? 1 : 0) + (rank < p.S - 1 ? 1 : 0));
+        ptx::mbar_arrive_expect_tx(ptx::smem_addr(sm.halo_bar + (blk & 1)), bytes);
+    }
+}
+
+// First step > 0 at which a local group restarts (INT_MAX if none); later
+// restarts follow every g steps.
+__device__ __forceinline__ int first_restart(int g, int L, bool fwd) {
+    if (g <= 0) return 0x7fffffff;
+    return fwd ? g : ((L - 1) % g) + 1;
+}
+
+// Per-step quantities of one position that do not depend on h: the scaled
+// products p_o of sigmoid denominators, the reciprocal of their sum, lambda*x
+// and u.
+struct StepW1 {
+    float p0, p1, p2, r, lx, u;
+};
+
+template <bool kRefine>
+__device__ __forceinline__ StepW1 prep_one(bool border, bool lo, bool hi, float x, float z0,
+                                           float z1, float z2, float lam, float u) {
+    StepW1 W;
+    W.lx = lam * x;
+    W.u = u;
+    const float kScale = 2.3283064365386963e-10f;  // 2^-32
+    float a0 = ex2_approx(fmaf(z0, -1.4426950408889634f, -32.0f)) + kScale;
+    const float a1 = ex2_approx(fmaf(z1, -1.4426950408889634f, -32.0f)) + kScale;
+    float a2 = ex2_approx(fmaf(z2, -1.4426950408889634f, -32.0f)) + kScale;
+    if (border) {  // a missing neighbour: a = scaled 1 (neutral), product p = 0
+        a0 = lo ? a0 : kScale;
+        a2 = hi ? a2 : kScale;
+    }
+    W.p0 = a1 * a2;
+    W.p1 = a0 * a2;
+    W.p2 = a0 * a1;
+    if (border) {
+        W.p0 = lo ? W.p0 : 0.0f;
+        W.p2 = hi ? W.p2 : 0.0f;
+    }
+    const float sum = W.p0 + W.p1 + W.p2;
+    W.r = rcp_approx(sum);
+    if (kRefine) W.r = fmaf(W.r, fmaf(-sum, W.r, 1.0f), W.r);
+    return W;
+}
+
+// The h-dependent part of a step:
+//   h = (p0*h_left + p1*h_self + p2*h_right) / (p0 + p1 + p2) + lambda*x.
+__device__ __forceinline__ float finish_one(const StepW1& W, float hl, float hs, float hr) {
+    return fmaf(fmaf(W.p2, hr, fmaf(W.p1, hs, W.p0 * hl)), W.r, W.lx);
+}
+
+// Scalar halo exchange (one position per thread) after the last step of block blk.
+// Senders push their exact state to a neighbour; halo threads replace theirs.
+__device__ __forceinline__ float halo_exchange1(const FusedParams& p, const SmemView& sm, Phases& ph,
+                                                int rank, int Kc, int blk, int L, float h) {
+    const int t = threadIdx.x;
+    const int par = blk & 1;
+    if (rank > 0 && t >= kHalo && t < 2 * kHalo) {  // first owned -> left neighbour's right halo
+        const uint32_t ra =
+            ptx::map_shared(ptx::smem_addr(sm.rx + (par * 2 + 1) * kHalo + (t - kHalo)), rank - 1);
+        const uint32_t rb = ptx::map_shared(ptx::smem_addr(sm.halo_bar + par), rank - 1);
+        ptx::st_async_f32(ra, h, rb);
+    }
+    if (rank < p.S - 1 && t >= Kc && t < Kc + kHalo) {  // last owned -> right neighbour's left halo
+        const uint32_t ra =
+            ptx::map_shared(ptx::smem_addr(sm.rx + (par * 2 + 0) * kHalo + (t - Kc)), rank + 1);
+        const uint32_t rb = ptx::map_shared(ptx::smem_addr(sm.halo_bar + par), rank + 1);
+        ptx::st_async_f32(ra, h, rb);
+    }
+    const bool recv_l = rank > 0 && t < kHalo;
+    const bool recv_r = rank < p.S - 1 && t >= kHalo + Kc && t < 2 * kHalo + Kc;
+    if (recv_l || recv_r || t == 0) {
+        wait_bar(p, ph, sm.halo_bar + par, (ph.halo >> par) & 1u, 3);
+        if (recv_l) h = ptx::lds_f32(ptx::smem_addr(sm.rx + (par * 2 + 0) * kHalo + t));
+        if (recv_r) h = ptx::lds_f32(ptx::smem_addr(sm.rx + (par * 2 + 1) * kHalo + (t - kHalo - Kc)));
+    }
+    if (t == 0) arm_halo_block(p, sm, rank, blk + 2, L);
+    ph.halo ^= 1u << par;
+    return h;
+}
+
+// Per-thread geometry of one chain segment (thread t <-> position kb + t).
+struct Geo1 {
+    int k;
+    bool work, in, own, lo, hi, border;
+};
+__device__ __forceinline__ Geo1 make_geo1(int kb, int k0, int Kc, int K, int np) {
+    Geo1 g;
+    const int t = threadIdx.x;
+    g.k = kb + t;
+    g.work = t < np;
+    g.in = g.k >= 0 && g.k < K;
+    g.own = g.work && g.in && g.k >= k0 && g.k < k0 + Kc;
+    g.lo = g.k > 0;
+    g.hi = g.k < K - 1;
+    const int w0 = kb + 32 * (t >> 5);  // first position of this warp
+    g.border = (w0 <= 0) || (w0 + 31 >= K - 1);
+    return g;
+}
+
+// The producer warp (the warp after the consumer threads) issues the chain's
+// stages into the ring.  It waits for a slot's release (empty barrier, one
+// consumer arrival per use) before reusing it and never joins the consumers'
+// per-step barrier, so the time a TMA instruction blocks its issuing warp is
+// hidden from the recurrence.  Lane 0 sets the expected bytes, lane b issues
+// box b (tensor b / nb, box b % nb).
+struct ProducerState {
+    uint32_t used;   // bit s: slot s has been filled before
+    uint32_t phase;  // bit s: parity of the next release of slot s
+    bool abort;
+};
+
+template <class BoxFn>
+__device__ __forceinline__ void producer_run(const FusedParams& p, const SmemView& sm,
+                                             ProducerState& ps, int nst, int nb,
+                                             uint32_t stage_bytes, BoxFn&& box) {
+    const int lane = threadIdx.x & 31;
+    for (int st = 0; st < nst; ++st) {
+        const int sl = st % p.stages;
+        if (ps.used & (1u << sl)) {
+            if (!ps.abort && !ptx::wait_parity_bounded(ptx::smem_addr(sm.empty_bar + sl),
+                                                       (ps.phase >> sl) & 1u, p.timeout_ns)) {
+                ps.abort = true;
+                report_error(p, 6);
+            }
+            ps.phase ^= 1u << sl;
+        }
+        ps.used |= 1u << sl;
+        const uint32_t bar = ptx::smem_addr(sm.full_bar + sl);
+        if (lane == 0) ptx::mbar_arrive_expect_tx(bar, stage_bytes);
+        __syncwarp();
+        if (lane < 6 * nb) box(st, sl, lane / nb, lane % nb, bar);
+        __syncwarp();
+    }
+}
+
+// Consumer side: thread 0 releases slot `sl` after a barrier that follows the
+// consumers' last read of it.
+__device__ __forceinline__ void release_slot(const SmemView& sm, int sl) {
+    if (threadIdx.x == 0) ptx::mbar_arrive(ptx::smem_addr(sm.empty_bar + sl));
+}
+
+__device__ __forceinline__ const CUtensorMap* tensor_map(const FusedParams& p, const CUtensorMap* xmap,
+                                                         int d, int tensor) {
+    return tensor == 0 ? xmap : tensor <= 3 ? &p.tm_z[d] : tensor == 4 ? &p.tm_l[d] : &p.tm_u[d];
+}
+__device__ __forceinline__ int tensor_z(int q, int tensor) {
+    return tensor == 0 ? q : tensor <= 3 ? 3 * q + tensor - 1 : q;
+}
+
+// Zero the two line buffers and arm the first two halo blocks.
+__device__ __forceinline__ void chain_begin(const FusedParams& p, const SmemView& sm, int rank,
+                                            int L) {
+    const int t = threadIdx.x;
+    for (int e = t; e < 2 * sm.line; e += blockDim.x) sm.hb[e] = 0.0f;
+    if (t == 0 && p.S > 1) {
+        arm_halo_block(p, sm, rank, 0, L);
+        arm_halo_block(p, sm, rank, 1, L);
+    }
+    __syncthreads();
+}
+
+template <class T>
+__device__ __forceinline__ float lds_elem(uint32_t a) {
+    if constexpr (sizeof(T) == 4)
+        return __uint_as_float(ptx::lds_u32(a));
+    else
+        return __uint_as_float(ptx::lds_u16(a) << 16);
+}
+
+// ---------------------------------------------------------------- vertical scans
+template <class T, bool kRefine, bool FWD>  // FWD: d = 0 (top->bottom), else d = 1
+__device__ __forceinline__ void chain_vertical(const FusedParams& p, const SmemView& sm,
+                                               Phases& ph, ProducerState& ps, int q, int rank,
+                                               int producer_warp, uint64_t pol_in,
+                                               uint64_t pol_acc) {
+    constexpr int d = FWD ? 0 : 1;
+    const int H = p.H, W = p.W, L = H, K = W;
+    const int Kc = p.Kc_v, np = p.np_v, R = p.R_v, bw = p.bw_v, nb = p.nb_v;
+    const int k0 = rank * Kc, kb = k0 - (p.S > 1 ? kHalo : 0);
+    const int t = threadIdx.x;
+    const int nthr = (np + 31) & ~31;
+    const int nst = (L + R - 1) / R;
+    const int S_ = p.S, stages = p.stages, g_len = p.g;
+    chain_begin(p, sm, rank, L);
+
+    if ((t >> 5) == producer_warp) {
+        producer_run(p, sm, ps, nst, nb, 6u * nb * bw * R * sizeof(T),
+                     [&](int st, int sl, int tensor, int b, uint32_t bar) {
+                         const int row0 = FWD ? st * R : H - R - st * R;
+                         const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) + b * p.box_v;
+                         const CUtensorMap* map = tensor_map(p, &p.tm_xv, d, tensor);
+                         if (tensor == 0)
+                             ptx::tma_load_3d_normal(dst, map, kb + b * bw, row0, tensor_z(q, tensor), bar);
+                         else
+                             ptx::tma_load_3d(dst, map, kb + b * bw, row0, tensor_z(q, tensor), bar, pol_in);
+                     });
+    } else if (t < nthr) {
+        const Geo1 g = make_geo1(kb, k0, Kc, K, np);
+        const int cb = g.work ? t / bw : 0;
+        const uint32_t col_byte = cb * p.box_v + (t - cb * bw) * (int)sizeof(T);
+        const uint32_t ring_s = ptx::smem_addr(sm.ring);
+        const uint32_t hb_s = ptx::smem_addr(sm.hb);
+        const uint32_t line_b = sm.line * 4;
+        const uint32_t tb = p.tile_bytes;
+        const uint32_t row_b = bw * (uint32_t)sizeof(T);
+        float* out = p.slots + (size_t)(q % p.n_slots) * H * W +
+                     (FWD ? 0 : (size_t)(H - 1) * W) + (g.own ? g.k : 0);
+        const ptrdiff_t out_step = FWD ? W : -W;
+
+        // prep state: stage / row inside the stage of the NEXT step to prepare
+        int pst = 0, pw = 0, psl = 0;
+        auto prep_next = [&]() -> StepW1 {
+            if (pw == 0) {
+                wait_bar(p, ph, sm.full_bar + psl, (ph.full >> psl) & 1u, 1);
+                ph.full ^= 1u << psl;
+            }
+            StepW1 Wt = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (g.work) {
+                const uint32_t a = ring_s + psl * 6 * tb + col_byte + (FWD ? pw : R - 1 - pw) * row_b;
+                Wt = prep_one<kRefine>(g.border, g.lo, g.hi, lds_elem<T>(a), lds_elem<T>(a + tb),
+                                       lds_elem<T>(a + 2 * tb), lds_elem<T>(a + 3 * tb),
+                                       lds_elem<T>(a + 4 * tb), lds_elem<T>(a + 5 * tb));
+            }
+            if (++pw == R) {
+                pw = 0;
+                ++pst;
+                psl = (psl + 1 == stages) ? 0 : psl + 1;
+            }
+            return Wt;
+        };
+
+        StepW1 Wt = prep_next();
+        float h = 0.0f;
+        int next_rs = first_restart(g_len, L, FWD);
+        int to_x = kHalo;
+        int rel = 0, rel_sl = 0;  // next stage to release and its slot
+        int rel_last = (R < L ? R : L) - 1;  // its last step
+        for (int i = 0; i < L; ++i) {
+            bool start = (i == 0);
+            if (i == next_rs) {
+                start = true;
+                next_rs += g_len;
+            }
+            if (i > 0) {
+                ptx::named_barrier(1, nthr);
+                if (rel_last < i) {  // every consumer has finished reading stage `rel`
+                    release_slot(sm, rel_sl);
+                    ++rel;
+                    rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
+                    rel_last = min(rel_last + R, L - 1);
+                }
+            }
+            const uint32_t hprev = hb_s + ((i - 1) & 1) * line_b;
+            const bool exch = S_ > 1 && --to_x == 0;
+            if (exch) to_x = kHalo;
+            if (g.work) {
+                h = start ? Wt.lx
+                          : finish_one(Wt, ptx::lds_f32(hprev + 4 * (t + 1)), h,
+                                       ptx::lds_f32(hprev + 4 * (t + 3)));
+                if (g.border && !g.in) h = 0.0f;
+                if (exch && i + 1 < L)
+                    h = halo_exchange1(p, sm, ph, rank, Kc, (i + 1) / kHalo - 1, L, h);
+                ptx::sts_f32(hb_s + (i & 1) * line_b + 4 * (t + 2), h);
+            } else if (exch && i + 1 < L) {
+                ph.halo ^= 1u << (((i + 1) / kHalo - 1) & 1);
+            }
+            if (g.own) ptx::red_add_f32(out, Wt.u * h, pol_acc);
+            out += out_step;
+            if (i + 1 < L) Wt = prep_next();
+        }
+        ptx::named_barrier(1, nthr);
+        for (; rel < nst; ++rel) {  // stages whose last read was in the final step
+            release_slot(sm, rel_sl);
+            rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
+        }
+        if (t == 0) {
+            sm.cell[2] = (int)ph.full;
+            sm.cell[3] = (int)ph.halo;
+        }
+    }
+    __syncthreads();
+}
+
+// -------------------------------------------------------------- horizontal scans
+// A thread keeps its 32-byte row segment of all six tensors for the stage in
+// registers and extracts one element per step.
+template <class T>
+__device__ __forceinline__ float seg_elem(const uint4 (&v)[2], int e) {
+    constexpr int per = 16 / sizeof(T);
+    return vec_elem<T>(v[e / per], e % per);
+}
+
+template <class T, bool kRefine, bool FWD>  // FWD: d = 2 (left->right), else d = 3
+__device__ __forceinline__ void chain_horizontal(const FusedParams& p, const SmemView& sm,
+                                                 Phases& ph, ProducerState& ps, int q, int rank,
+                                                 int producer_warp, uint64_t pol_in,
+                                                 uint64_t pol_acc) {
+    constexpr int J = 32 / sizeof(T);  // steps per stage: one 32-byte row segment
+    constexpr int d = FWD ? 2 : 3;
+    const int H = p.H, W = p.W, L = W, K = H;
+    const int Kc = p.Kc_h, np = p.np_h, bh = p.bh_h, nb = p.nb_h;
+    const int k0 = rank * Kc, kb = k0 - (p.S > 1 ? kHalo : 0);
+    const int t = threadIdx.x;
+    const int nthr = (np + 31) & ~31;
+    const int nst = L / J;
+    const int S_ = p.S, stages = p.stages, g_len = p.g;
+    chain_begin(p, sm, rank, L);
+
+    if ((t >> 5) == producer_warp) {
+        producer_run(p, sm, ps, nst, nb, 6u * nb * bh * 32u,
+                     [&](int st, int sl, int tensor, int b, uint32_t bar) {
+                         const int col0 = FWD ? st * J : W - J - st * J;
+                         const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) + b * bh * 32;
+                         ptx::tma_load_3d_normal(dst, tensor_map(p, &p.tm_xh, d, tensor), col0,
+                                                 kb + b * bh, tensor_z(q, tensor), bar);
+                     });
+    } else if (t < nthr) {
+        const Geo1 g = make_geo1(kb, k0, Kc, K, np);
+        float* row = p.slots + (size_t)(q % p.n_slots) * H * W + (size_t)(g.own ? g.k : 0) * W;
+        const uint32_t ring_s = ptx::smem_addr(sm.ring);
+        const uint32_t hb_s = ptx::smem_addr(sm.hb);
+        const uint32_t line_b = sm.line * 4;
+        const uint32_t tb = p.tile_bytes;
+        uint4 v[6][2];
+        int lsl = 0;  // slot of the next stage to load
+        auto load_stage = [&]() {
+            wait_bar(p, ph, sm.full_bar + lsl, (ph.full >> lsl) & 1u, 1);
+            ph.full ^= 1u << lsl;
+#pragma unroll
+            for (int k6 = 0; k6 < 6; ++k6) {
+                const uint32_t a = ring_s + (lsl * 6 + k6) * tb + 32 * t;
+                v[k6][0] = g.work ? ptx::lds_v4(a) : make_uint4(0, 0, 0, 0);
+                v[k6][1] = g.work ? ptx::lds_v4(a + 16) : make_uint4(0, 0, 0, 0);
+            }
+            lsl = (lsl + 1 == stages) ? 0 : lsl + 1;
+        };
+        auto prep = [&](int e) -> StepW1 {
+            return prep_one<kRefine>(g.border, g.lo, g.hi, seg_elem<T>(v[0], e),
+                                     seg_elem<T>(v[1], e), seg_elem<T>(v[2], e),
+                                     seg_elem<T>(v[3], e), seg_elem<T>(v[4], e),
+                                     seg_elem<T>(v[5], e));
+        };
+
+        load_stage();
+        StepW1 Wt = prep(FWD ? 0 : J - 1);
+        float h = 0.0f;
+        float acc[J];
+        int next_rs = first_restart(g_len, L, FWD);
+        int to_x = kHalo;
+        int i = 0;
+        int rel_sl = 0;  // slot of the next stage to release
+        for (int st = 0; st < nst; ++st) {
+            static_for<J>([&](auto wc) {
+                constexpr int w = decltype(wc)::value;
+                constexpr int e = FWD ? w : J - 1 - w;  // column offset inside the segment
+                bool start = (i == 0);
+                if (i == next_rs) {
+                    start = true;
+                    next_rs += g_len;
+                }
+                if (i > 0) {
+                    ptx::named_barrier(1, nthr);
+                    // stage st was read into registers before this barrier
+                    if (w == 0 || i == 1) {
+                        release_slot(sm, rel_sl);
+                        rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
+                    }
+                }
+                const uint32_t hprev = hb_s + ((i - 1) & 1) * line_b;
+                const bool exch = S_ > 1 && --to_x == 0;
+                if (exch) to_x = kHalo;
+                if (g.work) {
+                    h = start ? Wt.lx
+                              : finish_one(Wt, ptx::lds_f32(hprev + 4 * (t + 1)), h,
+                                           ptx::lds_f32(hprev + 4 * (t + 3)));
+                    if (g.border && !g.in) h = 0.0f;
+                    if (exch && i + 1 < L)
+                        h = halo_exchange1(p, sm, ph, rank, Kc, (i + 1) / kHalo - 1, L, h);
+                    ptx::sts_f32(hb_s + (i & 1) * line_b + 4 * (t + 2), h);
+                } else if (exch && i + 1 < L) {
+                    ph.halo ^= 1u << (((i + 1) / kHalo - 1) & 1);
+                }
+                acc[e] = Wt.u * h;
+                if constexpr (w + 1 < J) {
+                    Wt = prep(FWD ? w + 1 : J - 2 - w);
+                } else {
+                    if (st + 1 < nst) {
+                        load_stage();
+                        Wt = prep(FWD ? 0 : J - 1);
+                    }
+                }
+                ++i;
+            });
+            if (g.own) {
+                const int col0 = FWD ? st * J : W - J - st * J;
+#pragma unroll
+                for (int e = 0; e < J; e += 4)
+                    ptx::red_add_v4_f32_hint(row + col0 + e, acc[e], acc[e + 1], acc[e + 2],
+                                             acc[e + 3], pol_acc);
+            }
+        }
+        // every stage was released at its first step (stage 0 at step 1);
+        // only a one-step chain still holds its stage
+        if (L == 1) {
+            ptx::named_barrier(1, nthr);
+            release_slot(sm, rel_sl);
+        }
+        if (t == 0) {
+            sm.cell[2] = (int)ph.full;
+            sm.cell[3] = (int)ph.halo;
+        }
+    }
+    __syncthreads();
+}
+
+// Rounds the finished slot of plane q to the output dtype, writes y, re-zeroes
+// the slot.  CTA `rank` of the team takes a contiguous 1/S share.
+template <class T>
+__device__ __forceinline__ void convert_plane(const FusedParams& p, int q, int rank) {
+    const size_t HW = (size_t)p.H * p.W;
+    float* slot = p.slots + (size_t)(q % p.n_slots) * HW;
+    T* yq = static_cast<T*>(p.y) + (size_t)q * HW;
+    const size_t nvec = HW / 4;  // HW is a multiple of 4 (W * sizeof(T) % 16 == 0)
+    const size_t per = (nvec + p.S - 1) / p.S;
+    const size_t v0 = per * rank, v1 = min(nvec, v0 + per);
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (size_t v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
+        float4* sp = reinterpret_cast<float4*>(slot) + v;
+        const float4 a = __ldcg(sp);
+        __stcg(sp, zero);
+        if constexpr (sizeof(T) == 4) {
+            __stcs(reinterpret_cast<float4*>(yq) + v, a);
+        } else {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(a.z, a.w);
+            uint2 packed;
+            packed.x = *reinterpret_cast<uint32_t*>(&lo);
+            packed.y = *reinterpret_cast<uint32_t*>(&hi);
+            __stcs(reinterpret_cast<uint2*>(yq) + v, packed);
+        }
+    }
+}
+
+__device__ __forceinline__ void team_sync(int S) {
+    if (S > 1)
+        ptx::cluster_sync();
+    else
+        __syncthreads();
+}
+
+// Leader writes `v` into cell `c` of every CTA of the team.
+__device__ __forceinline__ void team_broadcast(const SmemView& sm, int S, int c, int v) {
+    if (S > 1) {
+        for (int r = 0; r < S; ++r)
+            ptx::st_cluster_s32(ptx::map_shared(ptx::smem_addr(sm.cell + c), r), v);
+    } else {
+        sm.cell[c] = v;
+    }
+}
+
+template <class T, bool kRefine>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+    fused_kernel(const __grid_constant__ FusedParams p) {
+    extern __shared__ __align__(128) char smem_raw[];
+    const SmemView sm = carve(smem_raw, p);
+    const int rank = p.S > 1 ? (int)ptx::cluster_ctarank() : 0;
+    const int t = threadIdx.x;
+
+    const int producer_warp = (blockDim.x >> 5) - 1;
+    if (t == 0) {
+        for (int s = 0; s < kMaxStages; ++s) {
+            ptx::mbar_init(ptx::smem_addr(sm.full_bar + s), 1);
+            ptx::mbar_init(ptx::smem_addr(sm.empty_bar + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) ptx::mbar_init(ptx::smem_addr(sm.halo_bar + s), 1);
+        sm.cell[2] = 0;
+        sm.cell[3] = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tensormap(&p.tm_xv);
+        ptx::prefetch_tensormap(&p.tm_xh);
+    }
+    team_sync(p.S);
+
+    const uint64_t pol_in = ptx::policy_evict_first();
+    const uint64_t pol_acc = ptx::policy_evict_last();
+    bool abort = false;
+    ProducerState ps{0u, 0u, false};
+
+    while (true) {
+        if (rank == 0 && t == 0) {
+            int it = -1;
+            if (ptx::ld_acquire_gpu(&p.ctrl->sticky_error) != 0) {
+                // a previous launch aborted: its slots may be dirty
+                atomicCAS(&p.ctrl->call_error, 0, 4);
+            } else if (ptx::ld_acquire_gpu(&p.ctrl->call_error) == 0) {
+                it = atomicAdd(&p.ctrl->next_item, 1);
+                if (it >= p.n_items) {
+                    it = -1;
+                } else {
+                    const int q = it / p.nd;
+                    const int s = q % p.n_slots;
+                    const int want = q / p.n_slots + (p.force_stale ? 1000000 : 0);
+                    if (ptx::ld_acquire_gpu(&p.ctrl->slot_epoch[s]) != want) {
+                        const uint64_t t0 = ptx::global_timer_ns();
+                        while (ptx::ld_acquire_gpu(&p.ctrl->slot_epoch[s]) != want) {
+                            if (ptx::ld_acquire_gpu(&p.ctrl->call_error) != 0 ||
+                                ptx::global_timer_ns() - t0 > p.timeout_ns) {
+                                report_error(p, 2);
+                                it = -1;
+                                break;
+                            }
+                            __nanosleep(256);
+                        }
+                    }
+                }
+            }
+            team_broadcast(sm, p.S, 0, it);
+        }
+        team_sync(p.S);
+        const int it = sm.cell[0];
+        if (it < 0) break;
+        const int q = it / p.nd;
+        const int d = p.d0 + it % p.nd;
+
+        Phases ph{(uint32_t)sm.cell[2], (uint32_t)sm.cell[3], abort};
+        if (d == 0)
+            chain_vertical<T, kRefine, true>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
+        else if (d == 1)
+            chain_vertical<T, kRefine, false>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
+        else if (d == 2)
+            chain_horizontal<T, kRefine, true>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
+        else
+            chain_horizontal<T, kRefine, false>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
+        abort = abort || ph.abort || ps.abort;
+
+        // Publish this chain, decide whether this team closes the plane.
+        __threadfence();
+        team_sync(p.S);
+        if (rank == 0 && t == 0) {
+            const int old = ptx::atom_add_acq_rel_gpu(p.plane_done + q, 1);
+            team_broadcast(sm, p.S, 1, (old == p.nd - 1) ? 1 : 0);
+        }
+        team_sync(p.S);
+        if (sm.cell[1]) {
+            convert_plane<T>(p, q, rank);
+            __threadfence();
+            team_sync(p.S);
+            if (rank == 0 && t == 0)
+                ptx::st_release_gpu(&p.ctrl->slot_epoch[q % p.n_slots], q / p.n_slots + 1);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int W, int H, int64_t depth, int box_x,
+                int box_y) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const size_t es = dtype == 0 ? 4 : 2;
+    cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)depth};
+    cuuint64_t strides[2] = {(cuuint64_t)(W * es), (cuuint64_t)((size_t)H * W * es)};
+    cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     3, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int round_up(int a, int b) { return (a + b - 1) / b * b; }
+
+// Geometry of one team size S; false if it does not fit.
+bool geometry_for(int S, int H, int W, int es, FusedPlan* gm) {
+    FusedPlan g;
+    memset(&g, 0, sizeof(g));
+    g.S = S;
+    g.T = S > 1 ? kHalo : 0;
+    if (S == 1) {
+        g.Kc_v = round_up(W, 8);
+        g.Kc_h = round_up(H, 8);
+        g.np_v = W;
+        g.np_h = H;
+    } else {
+        g.Kc_v = round_up((W + S - 1) / S, 8);
+        g.Kc_h = round_up((H + S - 1) / S, 8);
+        if (g.Kc_v < g.T || g.Kc_h < g.T) return false;
+        g.np_v = g.Kc_v + 2 * g.T;
+        g.np_h = g.Kc_h + 2 * g.T;
+    }
+    const int npmax = g.np_v > g.np_h ? g.np_v : g.np_h;
+    const int tv = round_up(g.np_v, 32), th = round_up(g.np_h, 32);
+    g.threads = (tv > th ? tv : th) + 32;  // consumers + the producer warp
+    if (g.threads > kMaxThreads) return false;
+    if (6 * ((g.np_v + 255) / 256) > 32 || 6 * ((g.np_h + 255) / 256) > 32) return false;
+    // horizontal tile: np_h rows x 32 bytes; box offsets 128-byte aligned (4 rows)
+    g.nb_h = (g.np_h + 255) / 256;
+    g.bh_h = round_up((g.np_h + g.nb_h - 1) / g.nb_h, 8);
+    if (g.bh_h > 256) return false;
+    const int tile_h = g.nb_h * g.bh_h * 32;
+    // vertical tile: R rows x np_v columns in boxes of <= 256 columns (multiple of 8)
+    g.nb_v = (g.np_v + 255) / 256;
+    g.bw_v = round_up((g.np_v + g.nb_v - 1) / g.nb_v, 8);
+    if (g.bw_v > 256) return false;
+    g.R_v = tile_h / (g.nb_v * g.bw_v * es);
+    if (g.R_v > 32) g.R_v = 32;
+    if (g.R_v < 4) g.R_v = 4;
+    g.box_v = round_up(g.bw_v * g.R_v * es, 128);
+    const int tile_v = g.nb_v * g.box_v;
+    g.tile_bytes = round_up(tile_h > tile_v ? tile_h : tile_v, 128);
+    size_t a, b, c;
+    g.stages = 0;
+    for (int st = kMaxStages; st >= 2; --st) {
+        g.smem = smem_layout(g.tile_bytes, st, npmax, &a, &b, &c);
+        if (g.smem <= 227 * 1024) {
+            g.stages = st;
+            break;
+        }
+    }
+    if (g.stages == 0) return false;
+    *gm = g;
+    return true;
+}
+
+template <class T, bool kRefine>
+cudaError_t set_attributes(const FusedPlan& fp) {
+    auto kernel = fused_kernel<T, kRefine>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fp.smem);
+    if (e == cudaSuccess && fp.S > 1)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return e;
+}
+
+void fill_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, const FusedPlan& fp,
+                 int clusters, cudaStream_t stream) {
+    memset(cfg, 0, sizeof(*cfg));
+    cfg->gridDim = dim3(clusters * fp.S, 1, 1);
+    cfg->blockDim = dim3(fp.threads, 1, 1);
+    cfg->dynamicSmemBytes = fp.smem;
+    cfg->stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = fp.S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg->attrs = attr;
+    cfg->numAttrs = 1;
+}
+
+template <class T, bool kRefine>
+int max_teams(const FusedPlan& fp) {
+    if (set_attributes<T, kRefine>(fp) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    fill_config(&cfg, attr, fp, 1, 0);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fused_kernel<T, kRefine>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+template <class T, bool kRefine>
+cudaError_t launch_typed(Problem& pb, const FusedPlan& fp, void* ws) {
+    cudaError_t e = set_attributes<T, kRefine>(fp);
+    if (e != cudaSuccess) return e;
+    const int H = (int)pb.H, W = (int)pb.W;
+    const int nd = pb.d1 - pb.d0;
+    constexpr int J = 32 / (int)sizeof(T);  // horizontal box: 32-byte row segments
+    FusedParams prm;
+    memset(&prm, 0, sizeof(prm));
+    const int64_t planes = pb.planes();
+    if (!encode_map(&prm.tm_xv, pb.x, pb.dtype, W, H, planes, fp.bw_v, fp.R_v) ||
+        !encode_map(&prm.tm_xh, pb.x, pb.dtype, W, H, planes, J, fp.bh_h))
+        return cudaErrorInvalidValue;
+    for (int d = pb.d0; d < pb.d1; ++d) {
+        const bool vert = d < 2;
+        const int bx = vert ? fp.bw_v : J;
+        const int by = vert ? fp.R_v : fp.bh_h;
+        if (!encode_map(&prm.tm_z[d], pb.z.p[d], pb.dtype, W, H, 3 * planes, bx, by) ||
+            !encode_map(&prm.tm_l[d], pb.lam.p[d], pb.dtype, W, H, planes, bx, by) ||
+            !encode_map(&prm.tm_u[d], pb.u.p[d], pb.dtype, W, H, planes, bx, by))
+            return cudaErrorInvalidValue;
+    }
+    char* base = static_cast<char*>(ws);
+    prm.y = pb.y;
+    prm.ctrl = reinterpret_cast<FusedCtrl*>(base);
+    prm.plane_done = reinterpret_cast<int*>(base + sizeof(FusedCtrl));
+    prm.slots = reinterpret_cast<float*>(base + fp.ctrl_bytes);
+    prm.timeout_ns = fp.timeout_ns;
+    prm.H = H;
+    prm.W = W;
+    prm.planes = (int)planes;
+    prm.g = (int)pb.g;
+    prm.d0 = pb.d0;
+    prm.nd = nd;
+    prm.S = fp.S;
+    prm.Kc_v = fp.Kc_v;
+    prm.Kc_h = fp.Kc_h;
+    prm.np_v = fp.np_v;
+    prm.np_h = fp.np_h;
+    prm.nb_v = fp.nb_v;
+    prm.bw_v = fp.bw_v;
+    prm.R_v = fp.R_v;
+    prm.box_v = fp.box_v;
+    prm.nb_h = fp.nb_h;
+    prm.bh_h = fp.bh_h;
+    prm.tile_bytes = fp.tile_bytes;
+    prm.stages = fp.stages;
+    prm.J_h = 32 / (int)sizeof(T);
+    prm.n_slots = fp.n_slots;
+    prm.n_items = (int)(planes * nd);
+    prm.force_stale = fp.force_stale;
+
+    // Reset the per-call part of the control block (not the sticky error).
+    e = cudaMemsetAsync(base + kCtrlResetOffset, 0, fp.ctrl_bytes - kCtrlResetOffset, pb.stream);
+    if (e != cudaSuccess) return e;
+    if (fp.zero_slots) {
+        e = cudaMemsetAsync(prm.slots, 0, fp.slot_bytes * fp.n_slots, pb.stream);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    fill_config(&cfg, attr, fp, fp.n_teams, pb.stream);
+    if (pb.ev_begin) cudaEventRecord(pb.ev_begin, pb.stream);
+    e = cudaLaunchKernelEx(&cfg, fused_kernel<T, kRefine>, prm);
+    if (pb.ev_end) cudaEventRecord(pb.ev_end, pb.stream);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t fused_ctrl_bytes(int64_t planes) {
+    return ((sizeof(FusedCtrl) + sizeof(int) * (size_t)planes) + 255) & ~(size_t)255;
+}
+
+bool fused_plan(const Problem& pb, FusedPlan* fp) {
+    const int es = pb.dtype == 0 ? 4 : 2;
+    if (pb.H > 0x7fffffff / pb.W) return false;
+    if ((pb.W * es) % 32 != 0) return false;  // whole 32-byte horizontal stages (and TMA strides)
+    if (pb.planes() * 3 > 0x7fffffffLL) return false;
+    const int H = (int)pb.H, W = (int)pb.W;
+    const int nd = pb.d1 - pb.d0;
+    const size_t slot_bytes = sizeof(float) * (size_t)H * W;
+    const size_t l2_budget = (size_t)80 << 20;
+    for (int S : {1, 2, 4, 8}) {
+        FusedPlan plan;
+        if (!geometry_for(S, H, W, es, &plan)) continue;
+        int teams = pb.dtype == 0 ? max_teams<float, true>(plan)
+                                  : max_teams<__nv_bfloat16, false>(plan);
+        if (teams <= 0) continue;
+        const int64_t items = pb.planes() * nd;
+        if (teams > items) teams = (int)items;
+        // planes that can be in flight at once, plus two for the ones closing
+        const int64_t want_slots = (teams + nd - 1) / nd + 2;
+        int64_t cap = (int64_t)(l2_budget / slot_bytes);
+        if (cap < 1) cap = 1;
+        int64_t slots = want_slots < cap ? want_slots : cap;
+        if (slots > kMaxSlots) slots = kMaxSlots;
+        if (slots > pb.planes()) slots = pb.planes();
+        // Prefer a larger team when the slot budget, not the SM count, would
+        // leave teams idle.
+        const bool starved = (int64_t)slots * nd < teams && S < 8;
+        if (starved) {
+            FusedPlan g2;
+            if (geometry_for(S * 2, H, W, es, &g2)) continue;
+        }
+        plan.n_teams = teams;
+        plan.n_slots = (int)slots;
+        plan.slot_bytes = slot_bytes;
+        plan.ctrl_bytes = fused_ctrl_bytes(pb.planes());
+        plan.ws_bytes = plan.ctrl_bytes + slot_bytes * (size_t)slots;
+        plan.timeout_ns = 4000000000ull;
+        plan.zero_slots = false;
+        plan.force_stale = 0;
+        *fp = plan;
+        return true;
+    }
+    return false;
+}
+
+cudaError_t launch_fused(Problem& pb, const FusedPlan& fp, void* ws, int* launches) {
+    pb.kernel_name = "fused_kernel";
+    if (getenv("GSPN_DEBUG_PLAN"))
+        fprintf(stderr,
+                "gspn fused plan: S=%d T=%d Kc_v=%d Kc_h=%d np_v=%d np_h=%d nb_v=%d bw_v=%d R_v=%d "
+                "box_v=%d nb_h=%d bh_h=%d tile=%d stages=%d threads=%d smem=%zu teams=%d slots=%d\n",
+                fp.S, fp.T, fp.Kc_v, fp.Kc_h, fp.np_v, fp.np_h, fp.nb_v, fp.bw_v, fp.R_v, fp.box_v,
+                fp.nb_h, fp.bh_h, fp.tile_bytes, fp.stages, fp.threads, fp.smem, fp.n_teams,
+                fp.n_slots);
+    cudaError_t e = pb.dtype == 0 ? launch_typed<float, true>(pb, fp, ws)
+                                  : launch_typed<__nv_bfloat16, false>(pb, fp, ws);
+    if (e == cudaSuccess) *launches += 1;
+    return e;
+}
+
+}  // namespace gspn

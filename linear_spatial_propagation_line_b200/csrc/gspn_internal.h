@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <string.h>
+
 #include "gspn_common.cuh"
 
 namespace gspn {
@@ -38,5 +40,24 @@ cudaError_t launch_small_plane(Problem& pb, int* launches);
 // workspace `ws` (B*C*H*W floats, zeroed here), then a conversion kernel
 // writes y.
 cudaError_t launch_chain(Problem& pb, float* ws, int* launches);
+
+// Fused persistent path (large planes whose rows are 16-byte multiples): one
+// launch computes all directions, accumulating in L2-resident fp32 slots.
+struct FusedPlan {
+    int S, T;                 // CTAs per team (cluster), halo width
+    int Kc_v, Kc_h, np_v, np_h;
+    int nb_v, bw_v, R_v, box_v, nb_h, bh_h;
+    int tile_bytes, threads, stages;
+    size_t smem;
+    int n_teams, n_slots;
+    size_t slot_bytes, ctrl_bytes, ws_bytes;
+    unsigned long long timeout_ns;
+    bool zero_slots;          // clear the slot area before the launch
+    int force_stale;          // test hook: make the slot wait expire
+};
+bool fused_plan(const Problem& pb, FusedPlan* fp);
+cudaError_t launch_fused(Problem& pb, const FusedPlan& fp, void* ws, int* launches);
+// Offset of the sticky device error word inside the fused workspace.
+constexpr size_t kFusedStickyErrorOffset = 0;
 
 }  // namespace gspn

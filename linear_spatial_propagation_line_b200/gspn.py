@@ -64,6 +64,10 @@ def load_library():
         lib.gspn_set_timing_events.restype = ci
         lib.gspn_last_kernel_name.argtypes = []
         lib.gspn_last_kernel_name.restype = ctypes.c_char_p
+        lib.gspn_check_device_status.argtypes = [vp]
+        lib.gspn_check_device_status.restype = ci
+        lib.gspn_debug_force_timeout.argtypes = [i64]
+        lib.gspn_debug_force_timeout.restype = ci
         _lib = lib
         return lib
 
@@ -100,6 +104,20 @@ def set_timing_events(begin=None, end=None):
 
 def last_kernel_name() -> str:
     return load_library().gspn_last_kernel_name().decode()
+
+
+def check_device_status(stream=None, device=None) -> int:
+    """Synchronise and return GSPN_OK (0) or GSPN_ERR_TIMEOUT (-7) if a bounded
+    device-side wait expired since the last check."""
+    lib = load_library()
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(device):
+        return lib.gspn_check_device_status(_stream_handle(device, stream))
+
+
+def debug_force_timeout(timeout_ns: int):
+    """Make the next large-plane launch on this thread expire a bounded wait."""
+    _check(load_library().gspn_debug_force_timeout(int(timeout_ns)))
 
 
 def release():

@@ -76,6 +76,45 @@ def test_shapes_global(H, W, dtype, cuda_device):
     check(wl, cuda_device, seed=H * 1000 + W)
 
 
+# Large planes on the fused kernel with multi-CTA teams (halo exchange through
+# DSMEM): 2-, 4- and 8-CTA teams, ragged owned ranges, local groups.
+TEAM_SHAPES = [(700, 96, 0), (96, 704, 0), (1500, 200, 0), (200, 1504, 0), (2100, 64, 0),
+               (3000, 256, 0), (1201, 160, 100), (160, 1208, 33), (1100, 1000, 0)]
+
+
+@pytest.mark.parametrize("H,W,g", TEAM_SHAPES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_large_planes_multi_cta_teams(H, W, g, dtype, cuda_device):
+    wl = Workload("team", 1, 2, H, W, g, dtype)
+    check(wl, cuda_device, seed=H + 7 * W + g)
+
+
+def test_forced_timeout_is_reported_and_recovers(cuda_device):
+    """A slot hand-over that never comes makes the kernel give up after its
+    bounded wait; the host sees GSPN_ERR_TIMEOUT and the next call is exact."""
+    wl = Workload("timeout", 1, 3, 256, 512, 0, "f32")
+    inp = inputs.make_inputs(wl, 6)
+    dev = to_dev(inp, cuda_device)
+    assert gspn.check_device_status() == 0
+    gspn.debug_force_timeout(50_000_000)  # 50 ms
+    gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0)
+    assert gspn.last_kernel_name() == "fused_kernel"
+    assert gspn.check_device_status() == -7
+    assert gspn.check_device_status() == 0
+    y = gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0)
+    ref = oracle.forward(inp["x"], inp["wlogit"], inp["lam"], inp["u"], 0)
+    assert rel_err(y, ref) <= TOL["f32"]
+    assert gspn.check_device_status() == 0
+
+
+def test_fused_path_is_used_for_the_headline_shape(cuda_device):
+    wl = WORKLOADS[inputs.HEADLINE].with_(C=2)
+    dev = to_dev(inputs.make_inputs(wl, 0), cuda_device)
+    gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0)
+    assert gspn.last_kernel_name() == "fused_kernel"
+    assert gspn.last_launch_count() == 1
+
+
 @pytest.mark.parametrize("H,W,g", [(28, 28, 7), (30, 27, 7), (16, 16, 1), (16, 16, 16),
                                    (16, 16, 100), (64, 64, 5), (130, 96, 7), (97, 200, 64),
                                    (300, 70, 1), (70, 300, 301)])
@@ -116,6 +155,7 @@ def test_large_plane_repeat_within_tolerance(cuda_device):
     a = gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0).double()
     b = gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0).double()
     assert float((a - b).abs().max() / a.abs().max()) <= 1e-6
+    assert gspn.check_device_status() == 0
 
 
 def test_host_entry_matches_device_entry(cuda_device):
