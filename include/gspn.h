@@ -71,6 +71,7 @@ extern "C" {
 #define GSPN_ERR_TIMEOUT (-7)  /* a bounded device-side wait gave up */
 #define GSPN_ERR_DIR (-8)      /* direction index outside 0..3 */
 #define GSPN_ERR_ALIAS (-9)    /* y overlaps an input */
+#define GSPN_ERR_SCRATCH (-10) /* B*C*H*W > GSPN_NOALLOC_MAX_ELEMENTS (gspn_forward_noalloc) */
 
 /*
  * Four-direction GSPN propagation (the operation above):
@@ -105,6 +106,33 @@ int gspn_forward_dir(const void* x, const void* wlogit, const void* lam, const v
 int gspn_forward_host(const void* x, const void* const wlogit[4], const void* const lam[4],
                       const void* const u[4], int64_t B, int64_t C, int64_t H, int64_t W,
                       int64_t group_len, int dtype, void* stream, void* y);
+
+/*
+ * gspn_forward without any device allocation.  The operation has no
+ * counterpart in the GSPN papers or pages: it is a deployment variant of the
+ * same computation for callers that cannot call cudaMalloc when they run it
+ * -- a process whose device memory is owned by another allocator (a caching
+ * allocator or a pool that reserved the GPU up front), or a latency-bound
+ * loop that cannot take the device-wide synchronisation of cudaMalloc /
+ * cudaFree.
+ *
+ * Same operation, arguments, layouts, alignment and errors as gspn_forward.
+ * It always runs the line-chain kernel (one CTA per plane and direction),
+ * accumulating in a fixed fp32 scratch array that is part of the library
+ * image (one per device) instead of an allocated workspace; the scratch is
+ * zeroed on `stream` at the start of every call.  Limit: B*C*H*W must not
+ * exceed GSPN_NOALLOC_MAX_ELEMENTS, else GSPN_ERR_SCRATCH with nothing
+ * launched.
+ *
+ * Concurrency: all calls on one device share that scratch, so calls must not
+ * overlap on the GPU -- issue them on one stream, or order them with events.
+ * The first call on each device looks the scratch up (and may load the
+ * library's device code); make it before any stream capture begins.
+ */
+#define GSPN_NOALLOC_MAX_ELEMENTS (((int64_t)1) << 23) /* 32 MiB of fp32 */
+int gspn_forward_noalloc(const void* x, const void* const wlogit[4], const void* const lam[4],
+                         const void* const u[4], int64_t B, int64_t C, int64_t H, int64_t W,
+                         int64_t group_len, int dtype, void* stream, void* y);
 
 /* Kernels launched by the most recent successful gspn_forward on this thread. */
 int gspn_last_launch_count(void);

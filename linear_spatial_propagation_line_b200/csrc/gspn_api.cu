@@ -281,6 +281,29 @@ int gspn_forward_host(const void* x, const void* const wlogit[4], const void* co
     return GSPN_OK;
 }
 
+int gspn_forward_noalloc(const void* x, const void* const wlogit[4], const void* const lam[4],
+                         const void* const u[4], int64_t B, int64_t C, int64_t H, int64_t W,
+                         int64_t group_len, int dtype, void* stream, void* y) {
+    gspn::Problem pb;
+    int s = validate(x, wlogit, lam, u, B, C, H, W, group_len, dtype, 0, 4, true, y, &pb);
+    if (s != GSPN_OK) return s;
+    if (pb.pixch() > gspn::kNoAllocMaxPixch) return GSPN_ERR_SCRATCH;
+    int dev;
+    if ((s = current_device(&dev)) != GSPN_OK) return s;
+    float* scratch = nullptr;
+    cudaError_t e = gspn::noalloc_scratch(dev, &scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    pb.stream = static_cast<cudaStream_t>(stream);
+    pb.ev_begin = t_ev_begin;
+    pb.ev_end = t_ev_end;
+    int launches = 0;
+    e = gspn::launch_chain(pb, scratch, &launches);  // zeroes scratch[0, B*C*H*W) first
+    if (e != cudaSuccess) return cuda_fail(e);
+    t_last_launches = launches;
+    t_last_kernel = pb.kernel_name;
+    return GSPN_OK;
+}
+
 int gspn_last_launch_count(void) { return t_last_launches; }
 
 int gspn_check_device_status(void* stream) {
@@ -358,6 +381,7 @@ const char* gspn_status_string(int status) {
         case GSPN_ERR_TIMEOUT: return "a bounded device-side wait timed out";
         case GSPN_ERR_DIR: return "direction outside 0..3";
         case GSPN_ERR_ALIAS: return "output overlaps an input";
+        case GSPN_ERR_SCRATCH: return "B*C*H*W exceeds the fixed scratch of gspn_forward_noalloc";
         default: return "unknown status";
     }
 }

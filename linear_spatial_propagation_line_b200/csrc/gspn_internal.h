@@ -7,6 +7,7 @@
 
 #include <string.h>
 
+#include "../../include/gspn.h"
 #include "gspn_common.cuh"
 
 namespace gspn {
@@ -40,6 +41,13 @@ cudaError_t launch_small_plane(Problem& pb, int* launches);
 // workspace `ws` (B*C*H*W floats, zeroed here), then a conversion kernel
 // writes y.
 cudaError_t launch_chain(Problem& pb, float* ws, int* launches);
+
+// Fixed-scratch variant of the line-chain path (gspn_forward_noalloc): the
+// fp32 accumulator is a static device array of kNoAllocMaxPixch floats.
+// noalloc_scratch returns its address on `device` (which must be current),
+// looking it up on the first call for that device.
+constexpr int64_t kNoAllocMaxPixch = GSPN_NOALLOC_MAX_ELEMENTS;
+cudaError_t noalloc_scratch(int device, float** scratch);
 
 // Fused persistent path (large planes whose rows are 16-byte multiples): one
 // launch computes all directions, accumulating in L2-resident fp32 slots.

@@ -18,6 +18,9 @@ GSPN_F32 = 0
 GSPN_BF16 = 1
 _DTYPES = {torch.float32: GSPN_F32, torch.bfloat16: GSPN_BF16}
 
+# Largest B*C*H*W of forward_noalloc (GSPN_NOALLOC_MAX_ELEMENTS).
+NOALLOC_MAX_ELEMENTS = 1 << 23
+
 _lock = threading.Lock()
 _lib = None
 
@@ -53,6 +56,9 @@ def load_library():
         lib.gspn_forward_host.argtypes = [vp, arr4, arr4, arr4, i64, i64, i64, i64, i64, ci, vp,
                                           vp]
         lib.gspn_forward_host.restype = ci
+        lib.gspn_forward_noalloc.argtypes = [vp, arr4, arr4, arr4, i64, i64, i64, i64, i64, ci,
+                                             vp, vp]
+        lib.gspn_forward_noalloc.restype = ci
         for name in ("gspn_last_launch_count", "gspn_release", "gspn_version"):
             getattr(lib, name).argtypes = []
             getattr(lib, name).restype = ci
@@ -174,6 +180,26 @@ def forward(x, wlogit, lam, u, group_len: int = 0, out=None, stream=None):
                                 arr4(*[t.data_ptr() for t in lam]),
                                 arr4(*[t.data_ptr() for t in u]), B, C, H, W, int(group_len),
                                 _DTYPES[x.dtype], st, y.data_ptr()))
+    return y
+
+
+def forward_noalloc(x, wlogit, lam, u, group_len: int = 0, out=None, stream=None):
+    """gspn_forward_noalloc: forward() without any device allocation inside
+    the library.  The accumulator is a fixed per-device array of
+    NOALLOC_MAX_ELEMENTS fp32 values, so B*C*H*W is limited to that, and calls
+    on one device must not overlap on the GPU.  Pass ``out`` to keep the call
+    itself free of allocations."""
+    lib = load_library()
+    B, C, H, W = _validate(x, wlogit, lam, u, range(4), "cuda")
+    y = torch.empty_like(x) if out is None else out
+    _validate(y, wlogit, lam, u, [], "cuda")
+    arr4 = ctypes.c_void_p * 4
+    with torch.cuda.device(x.device):
+        st = _stream_handle(x.device, stream)
+        _check(lib.gspn_forward_noalloc(x.data_ptr(), arr4(*[t.data_ptr() for t in wlogit]),
+                                        arr4(*[t.data_ptr() for t in lam]),
+                                        arr4(*[t.data_ptr() for t in u]), B, C, H, W,
+                                        int(group_len), _DTYPES[x.dtype], st, y.data_ptr()))
     return y
 
 
