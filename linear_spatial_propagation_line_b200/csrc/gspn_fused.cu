@@ -15,16 +15,22 @@
 //    so neighbouring CTAs exchange their edge states only every kHalo steps,
 //    through DSMEM `st.async` stores that complete transaction bytes on the
 //    receiver's mbarrier.
-//  * Each thread owns two adjacent positions and does the arithmetic on packed
-//    fp32 pairs (sm_100 f32x2 FMA/MUL/ADD), so every instruction but the
-//    exponentials and reciprocals serves two pixels.  The previous line lives
-//    in a double-buffered shared-memory line; one named barrier over the
-//    active warps per step.
-//  * Inputs stream through a kStages-deep shared-memory ring filled by TMA
-//    tensor loads (no multicast): vertical scans load R rows x (Kc + 2*kHalo)
-//    columns per stage; horizontal scans load (Kc + 2*kHalo) rows x 16 bytes,
-//    so each thread reads its two row segments with 16-byte shared loads and
-//    the scan runs along W with no transposition copy.
+//  * Each consumer thread owns one position.  The previous line lives in a
+//    double-buffered shared-memory line; one named barrier over the consumer
+//    warps separates two steps.  The weights are software-pipelined: in the
+//    interval between two barriers a thread finishes step i, completes the
+//    products and reciprocal of step i+1 and issues the exponentials of step
+//    i+2, so the dependent chain between barriers stays short.
+//  * Inputs stream through a 2-3 stage shared-memory ring filled by TMA tensor
+//    loads (no multicast) from a dedicated producer warp.  A stage is one
+//    32-byte segment of steps (16 bf16 or 8 fp32 lines): vertical scans load
+//    that many rows x (Kc + 2*kHalo) columns; horizontal scans load
+//    (Kc + 2*kHalo) rows x 32 bytes, and each thread copies its row segment
+//    to registers 16 bytes at a time, so the scan runs along W with no
+//    transposition.  The stage loop is unrolled at compile time and a halo
+//    block (32 steps) is a whole number of stages, so the exchange runs
+//    between stages.  Warps with no border position run a variant without
+//    border selects.
 //  * The four chains of a plane accumulate u_d * h_d into an fp32 "slot" kept
 //    L2-resident (evict_last reductions; streaming inputs use evict_first).
 //    The team that finishes a plane's last chain rounds the slot to the output
@@ -212,31 +218,45 @@ __device__ __forceinline__ int first_restart(int g, int L, bool fwd) {
     return fwd ? g : ((L - 1) % g) + 1;
 }
 
-// Per-step quantities of one position that do not depend on h: the scaled
-// products p_o of sigmoid denominators, the reciprocal of their sum, lambda*x
-// and u.
+// Weights of one position, computed in two pipelined halves so the dependent
+// chain between two step barriers stays short:
+//   begin:    a_o = 2^-32 (1 + exp(-z_o)) for the three neighbours, lambda*x, u
+//   complete: p_o = product of the other two a's (0 for a missing neighbour),
+//             r = 1 / (p_0 + p_1 + p_2)
+// so that h = (p_0 h_left + p_1 h_self + p_2 h_right) r + lambda*x.
+struct StepA {
+    float a0, a1, a2, lx, u;
+};
 struct StepW1 {
     float p0, p1, p2, r, lx, u;
 };
 
-template <bool kRefine>
-__device__ __forceinline__ StepW1 prep_one(bool border, bool lo, bool hi, float x, float z0,
-                                           float z1, float z2, float lam, float u) {
-    StepW1 W;
-    W.lx = lam * x;
-    W.u = u;
+template <bool kBorder>
+__device__ __forceinline__ StepA begin_prep(float x, float z0, float z1, float z2, float lam,
+                                            float u, bool lo, bool hi) {
     const float kScale = 2.3283064365386963e-10f;  // 2^-32
-    float a0 = ex2_approx(fmaf(z0, -1.4426950408889634f, -32.0f)) + kScale;
-    const float a1 = ex2_approx(fmaf(z1, -1.4426950408889634f, -32.0f)) + kScale;
-    float a2 = ex2_approx(fmaf(z2, -1.4426950408889634f, -32.0f)) + kScale;
-    if (border) {  // a missing neighbour: a = scaled 1 (neutral), product p = 0
-        a0 = lo ? a0 : kScale;
-        a2 = hi ? a2 : kScale;
+    StepA A;
+    A.lx = lam * x;
+    A.u = u;
+    A.a0 = ex2_approx(fmaf(z0, -1.4426950408889634f, -32.0f)) + kScale;
+    A.a1 = ex2_approx(fmaf(z1, -1.4426950408889634f, -32.0f)) + kScale;
+    A.a2 = ex2_approx(fmaf(z2, -1.4426950408889634f, -32.0f)) + kScale;
+    if (kBorder) {  // a missing neighbour: a = scaled 1 (neutral)
+        A.a0 = lo ? A.a0 : kScale;
+        A.a2 = hi ? A.a2 : kScale;
     }
-    W.p0 = a1 * a2;
-    W.p1 = a0 * a2;
-    W.p2 = a0 * a1;
-    if (border) {
+    return A;
+}
+
+template <bool kRefine, bool kBorder>
+__device__ __forceinline__ StepW1 complete_prep(const StepA& A, bool lo, bool hi) {
+    StepW1 W;
+    W.lx = A.lx;
+    W.u = A.u;
+    W.p0 = A.a1 * A.a2;
+    W.p1 = A.a0 * A.a2;
+    W.p2 = A.a0 * A.a1;
+    if (kBorder) {  // ... and product p = 0
         W.p0 = lo ? W.p0 : 0.0f;
         W.p2 = hi ? W.p2 : 0.0f;
     }
@@ -246,14 +266,13 @@ __device__ __forceinline__ StepW1 prep_one(bool border, bool lo, bool hi, float 
     return W;
 }
 
-// The h-dependent part of a step:
-//   h = (p0*h_left + p1*h_self + p2*h_right) / (p0 + p1 + p2) + lambda*x.
 __device__ __forceinline__ float finish_one(const StepW1& W, float hl, float hs, float hr) {
     return fmaf(fmaf(W.p2, hr, fmaf(W.p1, hs, W.p0 * hl)), W.r, W.lx);
 }
 
-// Scalar halo exchange (one position per thread) after the last step of block blk.
-// Senders push their exact state to a neighbour; halo threads replace theirs.
+// Halo exchange after the last step of block blk (one position per thread).
+// Senders push their exact state to a neighbour; halo threads return the
+// received state (others return h unchanged).
 __device__ __forceinline__ float halo_exchange1(const FusedParams& p, const SmemView& sm, Phases& ph,
                                                 int rank, int Kc, int blk, int L, float h) {
     const int t = threadIdx.x;
@@ -280,25 +299,6 @@ __device__ __forceinline__ float halo_exchange1(const FusedParams& p, const Smem
     if (t == 0) arm_halo_block(p, sm, rank, blk + 2, L);
     ph.halo ^= 1u << par;
     return h;
-}
-
-// Per-thread geometry of one chain segment (thread t <-> position kb + t).
-struct Geo1 {
-    int k;
-    bool work, in, own, lo, hi, border;
-};
-__device__ __forceinline__ Geo1 make_geo1(int kb, int k0, int Kc, int K, int np) {
-    Geo1 g;
-    const int t = threadIdx.x;
-    g.k = kb + t;
-    g.work = t < np;
-    g.in = g.k >= 0 && g.k < K;
-    g.own = g.work && g.in && g.k >= k0 && g.k < k0 + Kc;
-    g.lo = g.k > 0;
-    g.hi = g.k < K - 1;
-    const int w0 = kb + 32 * (t >> 5);  // first position of this warp
-    g.border = (w0 <= 0) || (w0 + 31 >= K - 1);
-    return g;
 }
 
 // The producer warp (the warp after the consumer threads) issues the chain's
@@ -343,12 +343,190 @@ __device__ __forceinline__ void release_slot(const SmemView& sm, int sl) {
     if (threadIdx.x == 0) ptx::mbar_arrive(ptx::smem_addr(sm.empty_bar + sl));
 }
 
-__device__ __forceinline__ const CUtensorMap* tensor_map(const FusedParams& p, const CUtensorMap* xmap,
-                                                         int d, int tensor) {
+__device__ __forceinline__ const CUtensorMap* tensor_map(const FusedParams& p,
+                                                         const CUtensorMap* xmap, int d,
+                                                         int tensor) {
     return tensor == 0 ? xmap : tensor <= 3 ? &p.tm_z[d] : tensor == 4 ? &p.tm_l[d] : &p.tm_u[d];
 }
 __device__ __forceinline__ int tensor_z(int q, int tensor) {
     return tensor == 0 ? q : tensor <= 3 ? 3 * q + tensor - 1 : q;
+}
+
+template <class T>
+__device__ __forceinline__ float lds_elem(uint32_t a) {
+    if constexpr (sizeof(T) == 4)
+        return __uint_as_float(ptx::lds_u32(a));
+    else
+        return __uint_as_float(ptx::lds_u16(a) << 16);
+}
+
+// Element e of a 32-byte row segment held as two 16-byte vectors.
+template <class T>
+__device__ __forceinline__ float seg_elem(const uint4 (&v)[2], int e) {
+    constexpr int per = 16 / sizeof(T);
+    return vec_elem<T>(v[e / per], e % per);
+}
+
+// ------------------------------------------------------------------- one chain
+// Runs one (plane, direction) chain segment on this CTA.  VERT: scan along H
+// (positions are columns; a stage holds kSeg rows of a column window, read
+// straight from the tile); otherwise scan along W (positions are rows; a
+// stage holds each row's 32-byte segment, copied to registers 16 bytes at a
+// time).  Every stage covers kSeg = 32 / sizeof(T) steps, so a halo block (32
+// steps) is a whole number of stages and the exchange runs between stages.
+// Horizontal chains need W to be a multiple of kSeg (every stage full).
+template <class T, bool kRefine, bool VERT, bool FWD, bool kBorder>
+__device__ __forceinline__ void chain_consume(const FusedParams& p, const SmemView& sm, Phases& ph,
+                                              int q, int rank, uint64_t pol_acc) {
+    constexpr int kSeg = 32 / sizeof(T);
+    constexpr int kPer = kSeg / 2;  // elements per 16-byte half segment
+    const int H = p.H, W = p.W;
+    const int L = VERT ? H : W, K = VERT ? W : H;
+    const int Kc = VERT ? p.Kc_v : p.Kc_h, np = VERT ? p.np_v : p.np_h;
+    const int k0 = rank * Kc, kb = k0 - (p.S > 1 ? kHalo : 0);
+    const int t = threadIdx.x;
+    const int nthr = (np + 31) & ~31;
+    const int nst = (L + kSeg - 1) / kSeg;
+    const int stages = p.stages, g_len = p.g;
+    const bool multi = p.S > 1;
+
+    const int k = kb + t;
+    const bool work = t < np;
+    const bool in = k >= 0 && k < K;
+    const bool own = work && in && k >= k0 && k < k0 + Kc;
+    const bool lo = k > 0, hi = k < K - 1;
+
+    const uint32_t ring_s = ptx::smem_addr(sm.ring);
+    const uint32_t hb_s = ptx::smem_addr(sm.hb);
+    const uint32_t line_b = sm.line * 4;
+    const uint32_t tb = p.tile_bytes;
+    // vertical: byte offset of this thread's column inside a tile
+    const int cb = (VERT && work) ? t / p.bw_v : 0;
+    const uint32_t col_byte = VERT ? (cb * p.box_v + (t - cb * p.bw_v) * (int)sizeof(T)) : 32u * t;
+    const uint32_t row_b = VERT ? p.bw_v * (uint32_t)sizeof(T) : 0u;
+    float* const slot = p.slots + (size_t)(q % p.n_slots) * H * W;
+    float* const out_row = slot + (size_t)(own ? k : 0) * W;                   // horizontal
+    float* out_px = slot + (FWD ? 0 : (size_t)(H - 1) * W) + (own ? k : 0);  // vertical
+    const ptrdiff_t out_step = FWD ? W : -W;
+
+    uint4 v[6];      // horizontal: one 16-byte half of this row's segment, every tensor
+    float acc[4];    // horizontal: u * h of four consecutive columns
+    int lsl = 0;     // slot of the next stage to acquire
+    int rel_sl = 0;  // slot of the next stage to release
+    int released = 0;
+    auto acquire = [&]() {
+        wait_bar(p, ph, sm.full_bar + lsl, (ph.full >> lsl) & 1u, 1);
+        ph.full ^= 1u << lsl;
+        lsl = (lsl + 1 == stages) ? 0 : lsl + 1;
+    };
+    auto release = [&]() {
+        release_slot(sm, rel_sl);
+        rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
+        ++released;
+    };
+    // horizontal: load logical half jl (steps jl*kPer ..) of the stage in slot sl
+    auto load_half = [&](int sl, int jl) {
+        const uint32_t a = ring_s + sl * 6 * tb + col_byte + 16u * (FWD ? jl : 1 - jl);
+#pragma unroll
+        for (int k6 = 0; k6 < 6; ++k6)
+            v[k6] = work ? ptx::lds_v4(a + k6 * tb) : make_uint4(0, 0, 0, 0);
+    };
+    // first half of the weights of step w (0 <= w < kSeg) of the stage in slot sl
+    auto begin_at = [&](int sl, int w) -> StepA {
+        if constexpr (VERT) {
+            const uint32_t a = ring_s + sl * 6 * tb + col_byte + (FWD ? w : kSeg - 1 - w) * row_b;
+            return begin_prep<kBorder>(lds_elem<T>(a), lds_elem<T>(a + tb), lds_elem<T>(a + 2 * tb),
+                                       lds_elem<T>(a + 3 * tb), lds_elem<T>(a + 4 * tb),
+                                       lds_elem<T>(a + 5 * tb), lo, hi);
+        } else {
+            const int e = FWD ? (w % kPer) : (kPer - 1 - (w % kPer));
+            return begin_prep<kBorder>(vec_elem<T>(v[0], e), vec_elem<T>(v[1], e),
+                                       vec_elem<T>(v[2], e), vec_elem<T>(v[3], e),
+                                       vec_elem<T>(v[4], e), vec_elem<T>(v[5], e), lo, hi);
+        }
+    };
+
+    // Software pipeline: Wt = weights of the step about to run, A = first half
+    // of the next step's.
+    int cur_sl = 0;
+    acquire();
+    if constexpr (!VERT) load_half(cur_sl, 0);
+    StepA A = begin_at(cur_sl, 0);
+    StepW1 Wt = complete_prep<kRefine, kBorder>(A, lo, hi);
+    A = begin_at(cur_sl, 1);
+    float h = 0.0f;
+    int next_rs = first_restart(g_len, L, FWD);
+    int i = 0;
+    for (int st = 0; st < nst; ++st) {
+        const int nxt_sl = (cur_sl + 1 == stages) ? 0 : cur_sl + 1;
+        static_for<kSeg>([&](auto wc) {
+            constexpr int w = decltype(wc)::value;
+            if (i < L) {
+                bool start = (i == 0);
+                if (i == next_rs) {
+                    start = true;
+                    next_rs += g_len;
+                }
+                if (i > 0) {
+                    ptx::named_barrier(1, nthr);
+                    // the barrier follows the last read of the current stage:
+                    // vertical reads row kSeg-1 at step kSeg-3, horizontal loads
+                    // its second half at step kPer-2
+                    if (w == (VERT ? kSeg - 2 : kPer - 1)) release();
+                }
+                const uint32_t hprev = hb_s + ((i - 1) & 1) * line_b;
+                if (work) {
+                    h = start ? Wt.lx
+                              : finish_one(Wt, ptx::lds_f32(hprev + 4 * (t + 1)), h,
+                                           ptx::lds_f32(hprev + 4 * (t + 3)));
+                    if (kBorder && !in) h = 0.0f;
+                    ptx::sts_f32(hb_s + (i & 1) * line_b + 4 * (t + 2), h);
+                }
+                if constexpr (VERT) {
+                    if (own) ptx::red_add_f32(out_px, Wt.u * h, pol_acc);
+                    out_px += out_step;
+                } else {
+                    acc[FWD ? (w & 3) : 3 - (w & 3)] = Wt.u * h;
+                    if ((w & 3) == 3 && own) {
+                        const int c0 = FWD ? st * kSeg + (w - 3) : W - st * kSeg - (w + 1);
+                        ptx::red_add_v4_f32_hint(out_row + c0, acc[0], acc[1], acc[2], acc[3],
+                                                 pol_acc);
+                    }
+                }
+                // advance: Wt <- complete(A); A <- begin(step w + 2)
+                Wt = complete_prep<kRefine, kBorder>(A, lo, hi);
+                if constexpr (w + 2 < kSeg) {
+                    if constexpr (!VERT && w + 2 == kPer) load_half(cur_sl, 1);
+                    A = begin_at(cur_sl, w + 2);
+                } else {
+                    if (st + 1 < nst) {
+                        if constexpr (w + 2 == kSeg) {  // first step of the next stage
+                            acquire();
+                            if constexpr (!VERT) load_half(nxt_sl, 0);
+                        }
+                        A = begin_at(nxt_sl, w + 2 - kSeg);
+                    }
+                }
+                ++i;
+            }
+        });
+        cur_sl = nxt_sl;
+        // halo exchange at the end of every 32-step block that has a successor
+        if (multi && ((st + 1) * kSeg) % kHalo == 0 && (st + 1) * kSeg < L) {
+            const float hx = halo_exchange1(p, sm, ph, rank, Kc, (st + 1) * kSeg / kHalo - 1, L, h);
+            if (work && hx != h) {
+                h = hx;
+                ptx::sts_f32(hb_s + ((i - 1) & 1) * line_b + 4 * (t + 2), h);
+            }
+        }
+    }
+    // release the stages still held (read in the last steps)
+    ptx::named_barrier(1, nthr);
+    while (released < nst) release();
+    if (t == 0) {
+        sm.cell[2] = (int)ph.full;
+        sm.cell[3] = (int)ph.halo;
+    }
 }
 
 // Zero the two line buffers and arm the first two halo blocks.
@@ -363,256 +541,52 @@ __device__ __forceinline__ void chain_begin(const FusedParams& p, const SmemView
     __syncthreads();
 }
 
-template <class T>
-__device__ __forceinline__ float lds_elem(uint32_t a) {
-    if constexpr (sizeof(T) == 4)
-        return __uint_as_float(ptx::lds_u32(a));
-    else
-        return __uint_as_float(ptx::lds_u16(a) << 16);
-}
-
-// ---------------------------------------------------------------- vertical scans
-template <class T, bool kRefine, bool FWD>  // FWD: d = 0 (top->bottom), else d = 1
-__device__ __forceinline__ void chain_vertical(const FusedParams& p, const SmemView& sm,
-                                               Phases& ph, ProducerState& ps, int q, int rank,
-                                               int producer_warp, uint64_t pol_in,
-                                               uint64_t pol_acc) {
-    constexpr int d = FWD ? 0 : 1;
-    const int H = p.H, W = p.W, L = H, K = W;
-    const int Kc = p.Kc_v, np = p.np_v, R = p.R_v, bw = p.bw_v, nb = p.nb_v;
-    const int k0 = rank * Kc, kb = k0 - (p.S > 1 ? kHalo : 0);
+template <class T, bool kRefine, bool VERT, bool FWD>
+__device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& sm, Phases& ph,
+                                          ProducerState& ps, int q, int rank, int producer_warp,
+                                          uint64_t pol_in, uint64_t pol_acc) {
+    constexpr int kSeg = 32 / sizeof(T);
+    constexpr int d = VERT ? (FWD ? 0 : 1) : (FWD ? 2 : 3);
+    const int H = p.H, W = p.W;
+    const int L = VERT ? H : W, K = VERT ? W : H;
+    const int Kc = VERT ? p.Kc_v : p.Kc_h, np = VERT ? p.np_v : p.np_h;
+    const int kb = rank * Kc - (p.S > 1 ? kHalo : 0);
     const int t = threadIdx.x;
     const int nthr = (np + 31) & ~31;
-    const int nst = (L + R - 1) / R;
-    const int S_ = p.S, stages = p.stages, g_len = p.g;
+    const int nst = (L + kSeg - 1) / kSeg;
     chain_begin(p, sm, rank, L);
-
     if ((t >> 5) == producer_warp) {
-        producer_run(p, sm, ps, nst, nb, 6u * nb * bw * R * sizeof(T),
-                     [&](int st, int sl, int tensor, int b, uint32_t bar) {
-                         const int row0 = FWD ? st * R : H - R - st * R;
-                         const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) + b * p.box_v;
-                         const CUtensorMap* map = tensor_map(p, &p.tm_xv, d, tensor);
-                         if (tensor == 0)
-                             ptx::tma_load_3d_normal(dst, map, kb + b * bw, row0, tensor_z(q, tensor), bar);
-                         else
-                             ptx::tma_load_3d(dst, map, kb + b * bw, row0, tensor_z(q, tensor), bar, pol_in);
-                     });
+        if constexpr (VERT) {
+            const int nb = p.nb_v, bw = p.bw_v;
+            producer_run(p, sm, ps, nst, nb, 6u * nb * bw * kSeg * sizeof(T),
+                         [&](int st, int sl, int tensor, int b, uint32_t bar) {
+                             const int row0 = FWD ? st * kSeg : H - kSeg - st * kSeg;
+                             const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) + b * p.box_v;
+                             const CUtensorMap* map = tensor_map(p, &p.tm_xv, d, tensor);
+                             if (tensor == 0)
+                                 ptx::tma_load_3d_normal(dst, map, kb + b * bw, row0,
+                                                         tensor_z(q, tensor), bar);
+                             else
+                                 ptx::tma_load_3d(dst, map, kb + b * bw, row0, tensor_z(q, tensor),
+                                                  bar, pol_in);
+                         });
+        } else {
+            const int nb = p.nb_h, bh = p.bh_h;
+            producer_run(p, sm, ps, nst, nb, 6u * nb * bh * 32u,
+                         [&](int st, int sl, int tensor, int b, uint32_t bar) {
+                             const int col0 = FWD ? st * kSeg : W - kSeg - st * kSeg;
+                             const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) + b * bh * 32;
+                             ptx::tma_load_3d_normal(dst, tensor_map(p, &p.tm_xh, d, tensor), col0,
+                                                     kb + b * bh, tensor_z(q, tensor), bar);
+                         });
+        }
     } else if (t < nthr) {
-        const Geo1 g = make_geo1(kb, k0, Kc, K, np);
-        const int cb = g.work ? t / bw : 0;
-        const uint32_t col_byte = cb * p.box_v + (t - cb * bw) * (int)sizeof(T);
-        const uint32_t ring_s = ptx::smem_addr(sm.ring);
-        const uint32_t hb_s = ptx::smem_addr(sm.hb);
-        const uint32_t line_b = sm.line * 4;
-        const uint32_t tb = p.tile_bytes;
-        const uint32_t row_b = bw * (uint32_t)sizeof(T);
-        float* out = p.slots + (size_t)(q % p.n_slots) * H * W +
-                     (FWD ? 0 : (size_t)(H - 1) * W) + (g.own ? g.k : 0);
-        const ptrdiff_t out_step = FWD ? W : -W;
-
-        // prep state: stage / row inside the stage of the NEXT step to prepare
-        int pst = 0, pw = 0, psl = 0;
-        auto prep_next = [&]() -> StepW1 {
-            if (pw == 0) {
-                wait_bar(p, ph, sm.full_bar + psl, (ph.full >> psl) & 1u, 1);
-                ph.full ^= 1u << psl;
-            }
-            StepW1 Wt = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (g.work) {
-                const uint32_t a = ring_s + psl * 6 * tb + col_byte + (FWD ? pw : R - 1 - pw) * row_b;
-                Wt = prep_one<kRefine>(g.border, g.lo, g.hi, lds_elem<T>(a), lds_elem<T>(a + tb),
-                                       lds_elem<T>(a + 2 * tb), lds_elem<T>(a + 3 * tb),
-                                       lds_elem<T>(a + 4 * tb), lds_elem<T>(a + 5 * tb));
-            }
-            if (++pw == R) {
-                pw = 0;
-                ++pst;
-                psl = (psl + 1 == stages) ? 0 : psl + 1;
-            }
-            return Wt;
-        };
-
-        StepW1 Wt = prep_next();
-        float h = 0.0f;
-        int next_rs = first_restart(g_len, L, FWD);
-        int to_x = kHalo;
-        int rel = 0, rel_sl = 0;  // next stage to release and its slot
-        int rel_last = (R < L ? R : L) - 1;  // its last step
-        for (int i = 0; i < L; ++i) {
-            bool start = (i == 0);
-            if (i == next_rs) {
-                start = true;
-                next_rs += g_len;
-            }
-            if (i > 0) {
-                ptx::named_barrier(1, nthr);
-                if (rel_last < i) {  // every consumer has finished reading stage `rel`
-                    release_slot(sm, rel_sl);
-                    ++rel;
-                    rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
-                    rel_last = min(rel_last + R, L - 1);
-                }
-            }
-            const uint32_t hprev = hb_s + ((i - 1) & 1) * line_b;
-            const bool exch = S_ > 1 && --to_x == 0;
-            if (exch) to_x = kHalo;
-            if (g.work) {
-                h = start ? Wt.lx
-                          : finish_one(Wt, ptx::lds_f32(hprev + 4 * (t + 1)), h,
-                                       ptx::lds_f32(hprev + 4 * (t + 3)));
-                if (g.border && !g.in) h = 0.0f;
-                if (exch && i + 1 < L)
-                    h = halo_exchange1(p, sm, ph, rank, Kc, (i + 1) / kHalo - 1, L, h);
-                ptx::sts_f32(hb_s + (i & 1) * line_b + 4 * (t + 2), h);
-            } else if (exch && i + 1 < L) {
-                ph.halo ^= 1u << (((i + 1) / kHalo - 1) & 1);
-            }
-            if (g.own) ptx::red_add_f32(out, Wt.u * h, pol_acc);
-            out += out_step;
-            if (i + 1 < L) Wt = prep_next();
-        }
-        ptx::named_barrier(1, nthr);
-        for (; rel < nst; ++rel) {  // stages whose last read was in the final step
-            release_slot(sm, rel_sl);
-            rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
-        }
-        if (t == 0) {
-            sm.cell[2] = (int)ph.full;
-            sm.cell[3] = (int)ph.halo;
-        }
-    }
-    __syncthreads();
-}
-
-// -------------------------------------------------------------- horizontal scans
-// A thread keeps its 32-byte row segment of all six tensors for the stage in
-// registers and extracts one element per step.
-template <class T>
-__device__ __forceinline__ float seg_elem(const uint4 (&v)[2], int e) {
-    constexpr int per = 16 / sizeof(T);
-    return vec_elem<T>(v[e / per], e % per);
-}
-
-template <class T, bool kRefine, bool FWD>  // FWD: d = 2 (left->right), else d = 3
-__device__ __forceinline__ void chain_horizontal(const FusedParams& p, const SmemView& sm,
-                                                 Phases& ph, ProducerState& ps, int q, int rank,
-                                                 int producer_warp, uint64_t pol_in,
-                                                 uint64_t pol_acc) {
-    constexpr int J = 32 / sizeof(T);  // steps per stage: one 32-byte row segment
-    constexpr int d = FWD ? 2 : 3;
-    const int H = p.H, W = p.W, L = W, K = H;
-    const int Kc = p.Kc_h, np = p.np_h, bh = p.bh_h, nb = p.nb_h;
-    const int k0 = rank * Kc, kb = k0 - (p.S > 1 ? kHalo : 0);
-    const int t = threadIdx.x;
-    const int nthr = (np + 31) & ~31;
-    const int nst = L / J;
-    const int S_ = p.S, stages = p.stages, g_len = p.g;
-    chain_begin(p, sm, rank, L);
-
-    if ((t >> 5) == producer_warp) {
-        producer_run(p, sm, ps, nst, nb, 6u * nb * bh * 32u,
-                     [&](int st, int sl, int tensor, int b, uint32_t bar) {
-                         const int col0 = FWD ? st * J : W - J - st * J;
-                         const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) + b * bh * 32;
-                         ptx::tma_load_3d_normal(dst, tensor_map(p, &p.tm_xh, d, tensor), col0,
-                                                 kb + b * bh, tensor_z(q, tensor), bar);
-                     });
-    } else if (t < nthr) {
-        const Geo1 g = make_geo1(kb, k0, Kc, K, np);
-        float* row = p.slots + (size_t)(q % p.n_slots) * H * W + (size_t)(g.own ? g.k : 0) * W;
-        const uint32_t ring_s = ptx::smem_addr(sm.ring);
-        const uint32_t hb_s = ptx::smem_addr(sm.hb);
-        const uint32_t line_b = sm.line * 4;
-        const uint32_t tb = p.tile_bytes;
-        uint4 v[6][2];
-        int lsl = 0;  // slot of the next stage to load
-        auto load_stage = [&]() {
-            wait_bar(p, ph, sm.full_bar + lsl, (ph.full >> lsl) & 1u, 1);
-            ph.full ^= 1u << lsl;
-#pragma unroll
-            for (int k6 = 0; k6 < 6; ++k6) {
-                const uint32_t a = ring_s + (lsl * 6 + k6) * tb + 32 * t;
-                v[k6][0] = g.work ? ptx::lds_v4(a) : make_uint4(0, 0, 0, 0);
-                v[k6][1] = g.work ? ptx::lds_v4(a + 16) : make_uint4(0, 0, 0, 0);
-            }
-            lsl = (lsl + 1 == stages) ? 0 : lsl + 1;
-        };
-        auto prep = [&](int e) -> StepW1 {
-            return prep_one<kRefine>(g.border, g.lo, g.hi, seg_elem<T>(v[0], e),
-                                     seg_elem<T>(v[1], e), seg_elem<T>(v[2], e),
-                                     seg_elem<T>(v[3], e), seg_elem<T>(v[4], e),
-                                     seg_elem<T>(v[5], e));
-        };
-
-        load_stage();
-        StepW1 Wt = prep(FWD ? 0 : J - 1);
-        float h = 0.0f;
-        float acc[J];
-        int next_rs = first_restart(g_len, L, FWD);
-        int to_x = kHalo;
-        int i = 0;
-        int rel_sl = 0;  // slot of the next stage to release
-        for (int st = 0; st < nst; ++st) {
-            static_for<J>([&](auto wc) {
-                constexpr int w = decltype(wc)::value;
-                constexpr int e = FWD ? w : J - 1 - w;  // column offset inside the segment
-                bool start = (i == 0);
-                if (i == next_rs) {
-                    start = true;
-                    next_rs += g_len;
-                }
-                if (i > 0) {
-                    ptx::named_barrier(1, nthr);
-                    // stage st was read into registers before this barrier
-                    if (w == 0 || i == 1) {
-                        release_slot(sm, rel_sl);
-                        rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
-                    }
-                }
-                const uint32_t hprev = hb_s + ((i - 1) & 1) * line_b;
-                const bool exch = S_ > 1 && --to_x == 0;
-                if (exch) to_x = kHalo;
-                if (g.work) {
-                    h = start ? Wt.lx
-                              : finish_one(Wt, ptx::lds_f32(hprev + 4 * (t + 1)), h,
-                                           ptx::lds_f32(hprev + 4 * (t + 3)));
-                    if (g.border && !g.in) h = 0.0f;
-                    if (exch && i + 1 < L)
-                        h = halo_exchange1(p, sm, ph, rank, Kc, (i + 1) / kHalo - 1, L, h);
-                    ptx::sts_f32(hb_s + (i & 1) * line_b + 4 * (t + 2), h);
-                } else if (exch && i + 1 < L) {
-                    ph.halo ^= 1u << (((i + 1) / kHalo - 1) & 1);
-                }
-                acc[e] = Wt.u * h;
-                if constexpr (w + 1 < J) {
-                    Wt = prep(FWD ? w + 1 : J - 2 - w);
-                } else {
-                    if (st + 1 < nst) {
-                        load_stage();
-                        Wt = prep(FWD ? 0 : J - 1);
-                    }
-                }
-                ++i;
-            });
-            if (g.own) {
-                const int col0 = FWD ? st * J : W - J - st * J;
-#pragma unroll
-                for (int e = 0; e < J; e += 4)
-                    ptx::red_add_v4_f32_hint(row + col0 + e, acc[e], acc[e + 1], acc[e + 2],
-                                             acc[e + 3], pol_acc);
-            }
-        }
-        // every stage was released at its first step (stage 0 at step 1);
-        // only a one-step chain still holds its stage
-        if (L == 1) {
-            ptx::named_barrier(1, nthr);
-            release_slot(sm, rel_sl);
-        }
-        if (t == 0) {
-            sm.cell[2] = (int)ph.full;
-            sm.cell[3] = (int)ph.halo;
-        }
+        const int w0 = kb + 32 * (t >> 5);  // first position of this warp
+        const bool border = (w0 <= 0) || (w0 + 31 >= K - 1);
+        if (border)
+            chain_consume<T, kRefine, VERT, FWD, true>(p, sm, ph, q, rank, pol_acc);
+        else
+            chain_consume<T, kRefine, VERT, FWD, false>(p, sm, ph, q, rank, pol_acc);
     }
     __syncthreads();
 }
@@ -728,13 +702,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
         Phases ph{(uint32_t)sm.cell[2], (uint32_t)sm.cell[3], abort};
         if (d == 0)
-            chain_vertical<T, kRefine, true>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
+            run_chain<T, kRefine, true, true>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
         else if (d == 1)
-            chain_vertical<T, kRefine, false>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
+            run_chain<T, kRefine, true, false>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
         else if (d == 2)
-            chain_horizontal<T, kRefine, true>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
+            run_chain<T, kRefine, false, true>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
         else
-            chain_horizontal<T, kRefine, false>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
+            run_chain<T, kRefine, false, false>(p, sm, ph, ps, q, rank, producer_warp, pol_in, pol_acc);
         abort = abort || ph.abort || ps.abort;
 
         // Publish this chain, decide whether this team closes the plane.
@@ -819,9 +793,7 @@ bool geometry_for(int S, int H, int W, int es, FusedPlan* gm) {
     g.nb_v = (g.np_v + 255) / 256;
     g.bw_v = round_up((g.np_v + g.nb_v - 1) / g.nb_v, 8);
     if (g.bw_v > 256) return false;
-    g.R_v = tile_h / (g.nb_v * g.bw_v * es);
-    if (g.R_v > 32) g.R_v = 32;
-    if (g.R_v < 4) g.R_v = 4;
+    g.R_v = 32 / es;  // one 32-byte row segment of steps, as horizontally
     g.box_v = round_up(g.bw_v * g.R_v * es, 128);
     const int tile_v = g.nb_v * g.box_v;
     g.tile_bytes = round_up(tile_h > tile_v ? tile_h : tile_v, 128);
