@@ -65,7 +65,7 @@ using ptx::f2;
 constexpr int kMaxStages = 3;
 constexpr int kMaxSlots = 64;
 constexpr int kHalo = 32;        // halo width == steps between exchanges
-constexpr int kMaxThreads = 640; // one position per consumer thread + one producer warp
+constexpr int kMaxThreads = 320; // two positions per consumer thread + one producer warp
 
 // Control block in global memory (the first bytes of the fused workspace).
 struct FusedCtrl {
@@ -95,12 +95,10 @@ struct __align__(64) FusedParams {
     int S;                 // team size (CTAs per cluster)
     int Kc_v, Kc_h;        // owned positions per CTA (vertical / horizontal scans)
     int np_v, np_h;        // positions handled per CTA (owned + halos)
-    int nb_v, bw_v, R_v;   // vertical: column boxes, box width, rows per stage
-    int box_v;             // bytes between vertical boxes in a tile (128-aligned)
+    int nb_v;              // vertical: 64-column boxes per stage (one per consumer warp)
     int nb_h, bh_h;        // horizontal: row boxes, box height (multiple of 8)
     int tile_bytes;        // one tensor's tile in one stage
     int stages;            // depth of the shared-memory ring (2 or 3)
-    int J_h;               // horizontal steps per stage (32-byte row segments)
     int n_slots;
     int n_items;
     int force_stale;       // test hook: expect a slot epoch that never comes
@@ -218,83 +216,138 @@ __device__ __forceinline__ int first_restart(int g, int L, bool fwd) {
     return fwd ? g : ((L - 1) % g) + 1;
 }
 
-// Weights of one position, computed in two pipelined halves so the dependent
-// chain between two step barriers stays short:
+// ------------------------------------------------------------------ pair math
+// A consumer thread owns two adjacent positions (k, k+1) of the line; their
+// values travel as packed fp32 pairs (position k in the low half).  A step's
+// weights are computed in two pipelined halves so the dependent chain between
+// two step barriers stays short:
 //   begin:    a_o = 2^-32 (1 + exp(-z_o)) for the three neighbours, lambda*x, u
 //   complete: p_o = product of the other two a's (0 for a missing neighbour),
 //             r = 1 / (p_0 + p_1 + p_2)
 // so that h = (p_0 h_left + p_1 h_self + p_2 h_right) r + lambda*x.
-struct StepA {
-    float a0, a1, a2, lx, u;
+struct PairA {
+    f2 a0, a1, a2, lx, u;
 };
-struct StepW1 {
-    float p0, p1, p2, r, lx, u;
+struct PairW {
+    f2 p0, p1, p2, r, lx, u;
+};
+// Which neighbours exist (only consulted in warps that touch a border).
+struct PairFlags {
+    bool lo0, hi0, lo1, hi1;  // position k: k-1, k+1 exist; position k+1: k, k+2 exist
+    bool in0, in1;            // the positions lie inside the plane
+};
+
+constexpr float kScale = 2.3283064365386963e-10f;  // 2^-32
+constexpr float kNegLog2e = -1.4426950408889634f;
+
+__device__ __forceinline__ f2 splat(float v) { return ptx::pk(v, v); }
+__device__ __forceinline__ float lo_of(f2 v) {
+    float a, b;
+    ptx::upk(v, a, b);
+    return a;
+}
+__device__ __forceinline__ float hi_of(f2 v) {
+    float a, b;
+    ptx::upk(v, a, b);
+    return b;
+}
+__device__ __forceinline__ f2 ex2_pair(f2 t) {
+    float a, b;
+    ptx::upk(t, a, b);
+    return ptx::pk(ex2_approx(a), ex2_approx(b));
+}
+__device__ __forceinline__ f2 sel_pair(f2 v, bool keep0, bool keep1, float other) {
+    float a, b;
+    ptx::upk(v, a, b);
+    return ptx::pk(keep0 ? a : other, keep1 ? b : other);
+}
+
+// The six inputs of one step for this thread's pair.
+struct PairIn {
+    f2 x, z0, z1, z2, lam, u;
 };
 
 template <bool kBorder>
-__device__ __forceinline__ StepA begin_prep(float x, float z0, float z1, float z2, float lam,
-                                            float u, bool lo, bool hi) {
-    const float kScale = 2.3283064365386963e-10f;  // 2^-32
-    StepA A;
-    A.lx = lam * x;
-    A.u = u;
-    A.a0 = ex2_approx(fmaf(z0, -1.4426950408889634f, -32.0f)) + kScale;
-    A.a1 = ex2_approx(fmaf(z1, -1.4426950408889634f, -32.0f)) + kScale;
-    A.a2 = ex2_approx(fmaf(z2, -1.4426950408889634f, -32.0f)) + kScale;
+__device__ __forceinline__ PairA begin_pair(const PairIn& in, const PairFlags& f) {
+    const f2 kL = splat(kNegLog2e), kO = splat(-32.0f), kS = splat(kScale);
+    PairA A;
+    A.lx = ptx::mul2(in.lam, in.x);
+    A.u = in.u;
+    A.a0 = ptx::add2(ex2_pair(ptx::fma2(in.z0, kL, kO)), kS);
+    A.a1 = ptx::add2(ex2_pair(ptx::fma2(in.z1, kL, kO)), kS);
+    A.a2 = ptx::add2(ex2_pair(ptx::fma2(in.z2, kL, kO)), kS);
     if (kBorder) {  // a missing neighbour: a = scaled 1 (neutral)
-        A.a0 = lo ? A.a0 : kScale;
-        A.a2 = hi ? A.a2 : kScale;
+        A.a0 = sel_pair(A.a0, f.lo0, f.lo1, kScale);
+        A.a2 = sel_pair(A.a2, f.hi0, f.hi1, kScale);
     }
     return A;
 }
 
 template <bool kRefine, bool kBorder>
-__device__ __forceinline__ StepW1 complete_prep(const StepA& A, bool lo, bool hi) {
-    StepW1 W;
+__device__ __forceinline__ PairW complete_pair(const PairA& A, const PairFlags& f) {
+    PairW W;
     W.lx = A.lx;
     W.u = A.u;
-    W.p0 = A.a1 * A.a2;
-    W.p1 = A.a0 * A.a2;
-    W.p2 = A.a0 * A.a1;
+    W.p0 = ptx::mul2(A.a1, A.a2);
+    W.p1 = ptx::mul2(A.a0, A.a2);
+    W.p2 = ptx::mul2(A.a0, A.a1);
     if (kBorder) {  // ... and product p = 0
-        W.p0 = lo ? W.p0 : 0.0f;
-        W.p2 = hi ? W.p2 : 0.0f;
+        W.p0 = sel_pair(W.p0, f.lo0, f.lo1, 0.0f);
+        W.p2 = sel_pair(W.p2, f.hi0, f.hi1, 0.0f);
     }
-    const float sum = W.p0 + W.p1 + W.p2;
-    W.r = rcp_approx(sum);
-    if (kRefine) W.r = fmaf(W.r, fmaf(-sum, W.r, 1.0f), W.r);
+    const f2 sum = ptx::add2(ptx::add2(W.p0, W.p1), W.p2);
+    float s0, s1;
+    ptx::upk(sum, s0, s1);
+    W.r = ptx::pk(rcp_approx(s0), rcp_approx(s1));
+    if (kRefine) {  // one Newton step: r += r (1 - s r)
+        const f2 e = ptx::fma2(ptx::mul2(sum, splat(-1.0f)), W.r, splat(1.0f));
+        W.r = ptx::fma2(W.r, e, W.r);
+    }
     return W;
 }
 
-__device__ __forceinline__ float finish_one(const StepW1& W, float hl, float hs, float hr) {
-    return fmaf(fmaf(W.p2, hr, fmaf(W.p1, hs, W.p0 * hl)), W.r, W.lx);
+// h of the pair from the left neighbour pair (positions k-2, k-1), the pair's
+// own previous state and the right neighbour pair (k+2, k+3).
+__device__ __forceinline__ f2 finish_pair(const PairW& W, float left, f2 hs, float right) {
+    const f2 hl = ptx::pk(left, lo_of(hs));
+    const f2 hr = ptx::pk(hi_of(hs), right);
+    return ptx::fma2(ptx::fma2(W.p2, hr, ptx::fma2(W.p1, hs, ptx::mul2(W.p0, hl))), W.r, W.lx);
 }
 
-// Halo exchange after the last step of block blk (one position per thread).
-// Senders push their exact state to a neighbour; halo threads return the
-// received state (others return h unchanged).
-__device__ __forceinline__ float halo_exchange1(const FusedParams& p, const SmemView& sm, Phases& ph,
-                                                int rank, int Kc, int blk, int L, float h) {
+__device__ __forceinline__ f2 bf16x2_pair(uint32_t w) {
+    return ptx::pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Halo exchange after the last step of block blk.  Senders push their exact
+// pair to a neighbour CTA; halo threads return the received pair (others
+// return h unchanged).  Window position of this thread's pair: 2 * threadIdx.x.
+__device__ __forceinline__ f2 halo_exchange(const FusedParams& p, const SmemView& sm, Phases& ph,
+                                            int rank, int Kc, int blk, int L, f2 h) {
     const int t = threadIdx.x;
+    const int pos = 2 * t;
     const int par = blk & 1;
-    if (rank > 0 && t >= kHalo && t < 2 * kHalo) {  // first owned -> left neighbour's right halo
+    float a, b;
+    ptx::upk(h, a, b);
+    if (rank > 0 && pos >= kHalo && pos < 2 * kHalo) {  // first owned -> left neighbour's right halo
         const uint32_t ra =
-            ptx::map_shared(ptx::smem_addr(sm.rx + (par * 2 + 1) * kHalo + (t - kHalo)), rank - 1);
+            ptx::map_shared(ptx::smem_addr(sm.rx + (par * 2 + 1) * kHalo + (pos - kHalo)), rank - 1);
         const uint32_t rb = ptx::map_shared(ptx::smem_addr(sm.halo_bar + par), rank - 1);
-        ptx::st_async_f32(ra, h, rb);
+        ptx::st_async_f32x2(ra, a, b, rb);
     }
-    if (rank < p.S - 1 && t >= Kc && t < Kc + kHalo) {  // last owned -> right neighbour's left halo
+    if (rank < p.S - 1 && pos >= Kc && pos < Kc + kHalo) {  // last owned -> right neighbour's left halo
         const uint32_t ra =
-            ptx::map_shared(ptx::smem_addr(sm.rx + (par * 2 + 0) * kHalo + (t - Kc)), rank + 1);
+            ptx::map_shared(ptx::smem_addr(sm.rx + (par * 2 + 0) * kHalo + (pos - Kc)), rank + 1);
         const uint32_t rb = ptx::map_shared(ptx::smem_addr(sm.halo_bar + par), rank + 1);
-        ptx::st_async_f32(ra, h, rb);
+        ptx::st_async_f32x2(ra, a, b, rb);
     }
-    const bool recv_l = rank > 0 && t < kHalo;
-    const bool recv_r = rank < p.S - 1 && t >= kHalo + Kc && t < 2 * kHalo + Kc;
+    const bool recv_l = rank > 0 && pos < kHalo;
+    const bool recv_r = rank < p.S - 1 && pos >= kHalo + Kc && pos < 2 * kHalo + Kc;
     if (recv_l || recv_r || t == 0) {
         wait_bar(p, ph, sm.halo_bar + par, (ph.halo >> par) & 1u, 3);
-        if (recv_l) h = ptx::lds_f32(ptx::smem_addr(sm.rx + (par * 2 + 0) * kHalo + t));
-        if (recv_r) h = ptx::lds_f32(ptx::smem_addr(sm.rx + (par * 2 + 1) * kHalo + (t - kHalo - Kc)));
+        uint2 v = make_uint2(0u, 0u);
+        if (recv_l) v = ptx::lds_v2(ptx::smem_addr(sm.rx + (par * 2 + 0) * kHalo + pos));
+        if (recv_r) v = ptx::lds_v2(ptx::smem_addr(sm.rx + (par * 2 + 1) * kHalo + (pos - kHalo - Kc)));
+        if (recv_l || recv_r) h = ptx::pk(__uint_as_float(v.x), __uint_as_float(v.y));
     }
     if (t == 0) arm_halo_block(p, sm, rank, blk + 2, L);
     ph.halo ^= 1u << par;
@@ -305,8 +358,8 @@ __device__ __forceinline__ float halo_exchange1(const FusedParams& p, const Smem
 // stages into the ring.  It waits for a slot's release (empty barrier, one
 // consumer arrival per use) before reusing it and never joins the consumers'
 // per-step barrier, so the time a TMA instruction blocks its issuing warp is
-// hidden from the recurrence.  Lane 0 sets the expected bytes, lane b issues
-// box b (tensor b / nb, box b % nb).
+// hidden from the recurrence.  Lane 0 sets the expected bytes; the boxes of a
+// stage (6 tensors x nb boxes) are spread over the lanes.
 struct ProducerState {
     uint32_t used;   // bit s: slot s has been filled before
     uint32_t phase;  // bit s: parity of the next release of slot s
@@ -332,7 +385,7 @@ __device__ __forceinline__ void producer_run(const FusedParams& p, const SmemVie
         const uint32_t bar = ptx::smem_addr(sm.full_bar + sl);
         if (lane == 0) ptx::mbar_arrive_expect_tx(bar, stage_bytes);
         __syncwarp();
-        if (lane < 6 * nb) box(st, sl, lane / nb, lane % nb, bar);
+        for (int b = lane; b < 6 * nb; b += 32) box(st, sl, b / nb, b % nb, bar);
         __syncwarp();
     }
 }
@@ -352,67 +405,62 @@ __device__ __forceinline__ int tensor_z(int q, int tensor) {
     return tensor == 0 ? q : tensor <= 3 ? 3 * q + tensor - 1 : q;
 }
 
-template <class T>
-__device__ __forceinline__ float lds_elem(uint32_t a) {
-    if constexpr (sizeof(T) == 4)
-        return __uint_as_float(ptx::lds_u32(a));
-    else
-        return __uint_as_float(ptx::lds_u16(a) << 16);
-}
-
-// Element e of a 32-byte row segment held as two 16-byte vectors.
-template <class T>
-__device__ __forceinline__ float seg_elem(const uint4 (&v)[2], int e) {
-    constexpr int per = 16 / sizeof(T);
-    return vec_elem<T>(v[e / per], e % per);
-}
-
 // ------------------------------------------------------------------- one chain
-// Runs one (plane, direction) chain segment on this CTA.  VERT: scan along H
-// (positions are columns; a stage holds kSeg rows of a column window, read
-// straight from the tile); otherwise scan along W (positions are rows; a
-// stage holds each row's 32-byte segment, copied to registers 16 bytes at a
-// time).  Every stage covers kSeg = 32 / sizeof(T) steps, so a halo block (32
-// steps) is a whole number of stages and the exchange runs between stages.
-// Horizontal chains need W to be a multiple of kSeg (every stage full).
-template <class T, bool kRefine, bool VERT, bool FWD, bool kBorder>
-__device__ __forceinline__ void chain_consume(const FusedParams& p, const SmemView& sm, Phases& ph,
-                                              int q, int rank, uint64_t pol_acc) {
+// Runs one (plane, direction) chain segment on this CTA, two positions per
+// consumer thread.  VERT: scan along H (positions are columns; a stage holds
+// kSeg rows of 64-column boxes, one box per warp, read straight from the
+// tile); otherwise scan along W (positions are rows; a stage holds each row's
+// 32-byte segment, copied to registers 16 bytes at a time).  Every stage
+// covers kSeg = 32 / sizeof(T) steps, so a halo block (32 steps) is a whole
+// number of stages and the exchange runs between stages.  Horizontal chains
+// need W to be a multiple of kSeg (every stage full); a vertical chain's last
+// stage may run past the plane on zero-filled rows, whose results are not
+// accumulated.
+// Not inlined: each of the sixteen variants gets its own register allocation
+// (inlined together into the kernel they would share one and spill).
+template <class T, bool kRefine, bool VERT, bool FWD, bool kBorder, bool kLocal>
+__device__ __noinline__ Phases chain_consume(const FusedParams& p, const SmemView sm, Phases ph,
+                                             int q, int rank, uint64_t pol_acc) {
     constexpr int kSeg = 32 / sizeof(T);
-    constexpr int kPer = kSeg / 2;  // elements per 16-byte half segment
+    constexpr int kPer = kSeg / 2;                   // steps per 16-byte half segment
+    constexpr uint32_t kRowB = 64u * sizeof(T);      // vertical box row pitch
+    constexpr uint32_t kBoxB = kRowB * kSeg;         // vertical box bytes (2 KB)
     const int H = p.H, W = p.W;
     const int L = VERT ? H : W, K = VERT ? W : H;
     const int Kc = VERT ? p.Kc_v : p.Kc_h, np = VERT ? p.np_v : p.np_h;
     const int k0 = rank * Kc, kb = k0 - (p.S > 1 ? kHalo : 0);
-    const int t = threadIdx.x;
-    const int nthr = (np + 31) & ~31;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int nthr = np >> 1;
     const int nst = (L + kSeg - 1) / kSeg;
     const int stages = p.stages, g_len = p.g;
     const bool multi = p.S > 1;
 
-    const int k = kb + t;
-    const bool work = t < np;
-    const bool in = k >= 0 && k < K;
-    const bool own = work && in && k >= k0 && k < k0 + Kc;
-    const bool lo = k > 0, hi = k < K - 1;
+    const int k = kb + 2 * t;
+    const bool own = k >= k0 && k < k0 + Kc && k < K;
+    const bool own1 = own && k + 1 < K;  // differs from own only at an odd K (horizontal)
+    PairFlags fl;
+    fl.lo0 = k > 0;
+    fl.hi0 = k + 1 < K;
+    fl.lo1 = k >= 0;
+    fl.hi1 = k + 2 < K;
+    fl.in0 = k >= 0 && k < K;
+    fl.in1 = k >= 0 && k + 1 < K;
 
     const uint32_t ring_s = ptx::smem_addr(sm.ring);
-    const uint32_t hb_s = ptx::smem_addr(sm.hb);
-    const uint32_t line_b = sm.line * 4;
     const uint32_t tb = p.tile_bytes;
-    // vertical: byte offset of this thread's column inside a tile
-    const int cb = (VERT && work) ? t / p.bw_v : 0;
-    const uint32_t col_byte = VERT ? (cb * p.box_v + (t - cb * p.bw_v) * (int)sizeof(T)) : 32u * t;
-    const uint32_t row_b = VERT ? p.bw_v * (uint32_t)sizeof(T) : 0u;
+    const uint32_t col_byte = VERT ? warp * kBoxB + lane * (2u * (uint32_t)sizeof(T)) : 64u * t;
+    // line buffers: this pair at index 2t+2; neighbours pairs at 2t and 2t+4
+    const uint32_t hb0 = ptx::smem_addr(sm.hb) + 8u * t;
+    const uint32_t hb1 = hb0 + sm.line * 4;
     float* const slot = p.slots + (size_t)(q % p.n_slots) * H * W;
     float* const out_row = slot + (size_t)(own ? k : 0) * W;                   // horizontal
     float* out_px = slot + (FWD ? 0 : (size_t)(H - 1) * W) + (own ? k : 0);  // vertical
     const ptrdiff_t out_step = FWD ? W : -W;
 
-    uint4 v[6];      // horizontal: one 16-byte half of this row's segment, every tensor
-    float acc[4];    // horizontal: u * h of four consecutive columns
-    int lsl = 0;     // slot of the next stage to acquire
-    int rel_sl = 0;  // slot of the next stage to release
+    uint4 v0[6], v1[6];  // horizontal: the current 16-byte half segment of rows k, k+1
+    float acc0[4], acc1[4];
+    int lsl = 0;         // slot of the next stage to acquire
+    int rel_sl = 0;      // slot of the next stage to release
     int released = 0;
     auto acquire = [&]() {
         wait_bar(p, ph, sm.full_bar + lsl, (ph.full >> lsl) & 1u, 1);
@@ -424,26 +472,43 @@ __device__ __forceinline__ void chain_consume(const FusedParams& p, const SmemVi
         rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
         ++released;
     };
+    auto tile_base = [&](int sl) -> uint32_t { return ring_s + sl * 6 * tb + col_byte; };
     // horizontal: load logical half jl (steps jl*kPer ..) of the stage in slot sl
     auto load_half = [&](int sl, int jl) {
-        const uint32_t a = ring_s + sl * 6 * tb + col_byte + 16u * (FWD ? jl : 1 - jl);
+        const uint32_t b = tile_base(sl) + 16u * (FWD ? jl : 1 - jl);
 #pragma unroll
-        for (int k6 = 0; k6 < 6; ++k6)
-            v[k6] = work ? ptx::lds_v4(a + k6 * tb) : make_uint4(0, 0, 0, 0);
+        for (int k6 = 0; k6 < 6; ++k6) {
+            v0[k6] = ptx::lds_v4(b + k6 * tb);
+            v1[k6] = ptx::lds_v4(b + k6 * tb + 32u);
+        }
     };
-    // first half of the weights of step w (0 <= w < kSeg) of the stage in slot sl
-    auto begin_at = [&](int sl, int w) -> StepA {
+    // inputs of step w (0 <= w < kSeg) of the stage in slot sl
+    auto fetch = [&](int sl, int w) -> PairIn {
+        PairIn in;
+        f2 r[6];
         if constexpr (VERT) {
-            const uint32_t a = ring_s + sl * 6 * tb + col_byte + (FWD ? w : kSeg - 1 - w) * row_b;
-            return begin_prep<kBorder>(lds_elem<T>(a), lds_elem<T>(a + tb), lds_elem<T>(a + 2 * tb),
-                                       lds_elem<T>(a + 3 * tb), lds_elem<T>(a + 4 * tb),
-                                       lds_elem<T>(a + 5 * tb), lo, hi);
+            const uint32_t b = tile_base(sl) + (FWD ? w : kSeg - 1 - w) * kRowB;
+#pragma unroll
+            for (int k6 = 0; k6 < 6; ++k6) {
+                if constexpr (sizeof(T) == 4) {
+                    const uint2 u2 = ptx::lds_v2(b + k6 * tb);
+                    r[k6] = ptx::pk(__uint_as_float(u2.x), __uint_as_float(u2.y));
+                } else {
+                    r[k6] = bf16x2_pair(ptx::lds_u32(b + k6 * tb));
+                }
+            }
         } else {
             const int e = FWD ? (w % kPer) : (kPer - 1 - (w % kPer));
-            return begin_prep<kBorder>(vec_elem<T>(v[0], e), vec_elem<T>(v[1], e),
-                                       vec_elem<T>(v[2], e), vec_elem<T>(v[3], e),
-                                       vec_elem<T>(v[4], e), vec_elem<T>(v[5], e), lo, hi);
+#pragma unroll
+            for (int k6 = 0; k6 < 6; ++k6) r[k6] = ptx::pk(vec_elem<T>(v0[k6], e), vec_elem<T>(v1[k6], e));
         }
+        in.x = r[0];
+        in.z0 = r[1];
+        in.z1 = r[2];
+        in.z2 = r[3];
+        in.lam = r[4];
+        in.u = r[5];
+        return in;
     };
 
     // Software pipeline: Wt = weights of the step about to run, A = first half
@@ -451,72 +516,102 @@ __device__ __forceinline__ void chain_consume(const FusedParams& p, const SmemVi
     int cur_sl = 0;
     acquire();
     if constexpr (!VERT) load_half(cur_sl, 0);
-    StepA A = begin_at(cur_sl, 0);
-    StepW1 Wt = complete_prep<kRefine, kBorder>(A, lo, hi);
-    A = begin_at(cur_sl, 1);
-    float h = 0.0f;
+    PairW Wt = complete_pair<kRefine, kBorder>(begin_pair<kBorder>(fetch(cur_sl, 0), fl), fl);
+    PairA A = begin_pair<kBorder>(fetch(cur_sl, 1), fl);
+    f2 h = splat(0.0f);
     int next_rs = first_restart(g_len, L, FWD);
-    int i = 0;
     for (int st = 0; st < nst; ++st) {
         const int nxt_sl = (cur_sl + 1 == stages) ? 0 : cur_sl + 1;
+        const bool more = st + 1 < nst;
+        const int wlim = more ? kSeg : L - st * kSeg;  // vertical: steps inside the plane
         static_for<kSeg>([&](auto wc) {
             constexpr int w = decltype(wc)::value;
-            if (i < L) {
-                bool start = (i == 0);
-                if (i == next_rs) {
+            bool start = false;
+            if constexpr (w == 0) start = (st == 0);
+            if constexpr (kLocal) {
+                if (st * kSeg + w == next_rs) {
                     start = true;
                     next_rs += g_len;
                 }
-                if (i > 0) {
-                    ptx::named_barrier(1, nthr);
-                    // the barrier follows the last read of the current stage:
-                    // vertical reads row kSeg-1 at step kSeg-3, horizontal loads
-                    // its second half at step kPer-2
-                    if (w == (VERT ? kSeg - 2 : kPer - 1)) release();
+            }
+            if (w > 0 || st > 0) {
+                ptx::named_barrier(1, nthr);
+                // the barrier follows the last read of the current stage:
+                // vertical fetches row kSeg-1 at step kSeg-3, horizontal loads
+                // its second half at step kPer-2
+                if constexpr (w == (VERT ? kSeg - 2 : kPer - 1)) release();
+            }
+            const uint32_t hprev = (w & 1) ? hb0 : hb1;
+            const uint32_t hcur = (w & 1) ? hb1 : hb0;
+            // 1. neighbour state (the critical path)
+            const uint2 lp = ptx::lds_v2(hprev);
+            const uint2 rp = ptx::lds_v2(hprev + 16u);
+            // 2. shared-memory inputs of step w + 2 (vertical: six loads;
+            //    horizontal: the next half segment when step w + 2 starts one)
+            constexpr bool kNext = w + 2 >= kSeg;     // step w + 2 is in the next stage
+            constexpr int w2 = kNext ? w + 2 - kSeg : w + 2;
+            const bool have2 = !kNext || more;
+            const int sl2 = kNext ? nxt_sl : cur_sl;
+            if constexpr (kNext && w2 == 0) {
+                if (more) {
+                    acquire();
+                    if constexpr (!VERT) load_half(nxt_sl, 0);
                 }
-                const uint32_t hprev = hb_s + ((i - 1) & 1) * line_b;
-                if (work) {
-                    h = start ? Wt.lx
-                              : finish_one(Wt, ptx::lds_f32(hprev + 4 * (t + 1)), h,
-                                           ptx::lds_f32(hprev + 4 * (t + 3)));
-                    if (kBorder && !in) h = 0.0f;
-                    ptx::sts_f32(hb_s + (i & 1) * line_b + 4 * (t + 2), h);
+            }
+            if constexpr (!VERT && !kNext && w2 == kPer) load_half(cur_sl, 1);
+            PairIn in2;
+            if constexpr (VERT) {
+                if (have2) in2 = fetch(sl2, w2);
+            }
+            // 3. this step's state
+            f2 hn = start ? Wt.lx
+                          : finish_pair(Wt, __uint_as_float(lp.y), h, __uint_as_float(rp.x));
+            if (kBorder) hn = sel_pair(hn, fl.in0, fl.in1, 0.0f);
+            h = hn;
+            {
+                float a, b;
+                ptx::upk(h, a, b);
+                ptx::sts_v2_f32(hcur + 8u, a, b);
+            }
+            const f2 uh = ptx::mul2(Wt.u, h);
+            if constexpr (VERT) {
+                if (own && w < wlim) {
+                    float a, b;
+                    ptx::upk(uh, a, b);
+                    ptx::red_add_v2_f32(out_px, a, b, pol_acc);
                 }
-                if constexpr (VERT) {
-                    if (own) ptx::red_add_f32(out_px, Wt.u * h, pol_acc);
-                    out_px += out_step;
-                } else {
-                    acc[FWD ? (w & 3) : 3 - (w & 3)] = Wt.u * h;
-                    if ((w & 3) == 3 && own) {
-                        const int c0 = FWD ? st * kSeg + (w - 3) : W - st * kSeg - (w + 1);
-                        ptx::red_add_v4_f32_hint(out_row + c0, acc[0], acc[1], acc[2], acc[3],
+                out_px += out_step;
+            } else {
+                float a, b;
+                ptx::upk(uh, a, b);
+                acc0[FWD ? (w & 3) : 3 - (w & 3)] = a;
+                acc1[FWD ? (w & 3) : 3 - (w & 3)] = b;
+                if constexpr ((w & 3) == 3) {
+                    const int c0 = FWD ? st * kSeg + (w - 3) : W - st * kSeg - (w + 1);
+                    if (own)
+                        ptx::red_add_v4_f32_hint(out_row + c0, acc0[0], acc0[1], acc0[2], acc0[3],
                                                  pol_acc);
-                    }
+                    if (own1)
+                        ptx::red_add_v4_f32_hint(out_row + W + c0, acc1[0], acc1[1], acc1[2],
+                                                 acc1[3], pol_acc);
                 }
-                // advance: Wt <- complete(A); A <- begin(step w + 2)
-                Wt = complete_prep<kRefine, kBorder>(A, lo, hi);
-                if constexpr (w + 2 < kSeg) {
-                    if constexpr (!VERT && w + 2 == kPer) load_half(cur_sl, 1);
-                    A = begin_at(cur_sl, w + 2);
-                } else {
-                    if (st + 1 < nst) {
-                        if constexpr (w + 2 == kSeg) {  // first step of the next stage
-                            acquire();
-                            if constexpr (!VERT) load_half(nxt_sl, 0);
-                        }
-                        A = begin_at(nxt_sl, w + 2 - kSeg);
-                    }
-                }
-                ++i;
+            }
+            // 4. weights of step w + 1, first half of step w + 2's
+            Wt = complete_pair<kRefine, kBorder>(A, fl);
+            if (have2) {
+                if constexpr (!VERT) in2 = fetch(sl2, w2);
+                A = begin_pair<kBorder>(in2, fl);
             }
         });
         cur_sl = nxt_sl;
         // halo exchange at the end of every 32-step block that has a successor
         if (multi && ((st + 1) * kSeg) % kHalo == 0 && (st + 1) * kSeg < L) {
-            const float hx = halo_exchange1(p, sm, ph, rank, Kc, (st + 1) * kSeg / kHalo - 1, L, h);
-            if (work && hx != h) {
+            const f2 hx = halo_exchange(p, sm, ph, rank, Kc, (st + 1) * kSeg / kHalo - 1, L, h);
+            if (hx != h) {
                 h = hx;
-                ptx::sts_f32(hb_s + ((i - 1) & 1) * line_b + 4 * (t + 2), h);
+                float a, b;
+                ptx::upk(h, a, b);
+                ptx::sts_v2_f32(hb1 + 8u, a, b);  // the last step (odd) wrote line 1
             }
         }
     }
@@ -527,6 +622,7 @@ __device__ __forceinline__ void chain_consume(const FusedParams& p, const SmemVi
         sm.cell[2] = (int)ph.full;
         sm.cell[3] = (int)ph.halo;
     }
+    return ph;
 }
 
 // Zero the two line buffers and arm the first two halo blocks.
@@ -541,6 +637,16 @@ __device__ __forceinline__ void chain_begin(const FusedParams& p, const SmemView
     __syncthreads();
 }
 
+template <class T, bool kRefine, bool VERT, bool FWD, bool kBorder>
+__device__ __forceinline__ void consume_dispatch(const FusedParams& p, const SmemView& sm,
+                                                 Phases& ph, int q, int rank, uint64_t pol_acc,
+                                                 bool local) {
+    if (local)
+        ph = chain_consume<T, kRefine, VERT, FWD, kBorder, true>(p, sm, ph, q, rank, pol_acc);
+    else
+        ph = chain_consume<T, kRefine, VERT, FWD, kBorder, false>(p, sm, ph, q, rank, pol_acc);
+}
+
 template <class T, bool kRefine, bool VERT, bool FWD>
 __device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& sm, Phases& ph,
                                           ProducerState& ps, int q, int rank, int producer_warp,
@@ -552,22 +658,23 @@ __device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& 
     const int Kc = VERT ? p.Kc_v : p.Kc_h, np = VERT ? p.np_v : p.np_h;
     const int kb = rank * Kc - (p.S > 1 ? kHalo : 0);
     const int t = threadIdx.x;
-    const int nthr = (np + 31) & ~31;
+    const int nthr = np >> 1;
     const int nst = (L + kSeg - 1) / kSeg;
     chain_begin(p, sm, rank, L);
     if ((t >> 5) == producer_warp) {
         if constexpr (VERT) {
-            const int nb = p.nb_v, bw = p.bw_v;
-            producer_run(p, sm, ps, nst, nb, 6u * nb * bw * kSeg * sizeof(T),
+            const int nb = p.nb_v;
+            producer_run(p, sm, ps, nst, nb, 6u * nb * 64u * kSeg * sizeof(T),
                          [&](int st, int sl, int tensor, int b, uint32_t bar) {
                              const int row0 = FWD ? st * kSeg : H - kSeg - st * kSeg;
-                             const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) + b * p.box_v;
+                             const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) +
+                                                  b * (64u * kSeg * (uint32_t)sizeof(T));
                              const CUtensorMap* map = tensor_map(p, &p.tm_xv, d, tensor);
                              if (tensor == 0)
-                                 ptx::tma_load_3d_normal(dst, map, kb + b * bw, row0,
+                                 ptx::tma_load_3d_normal(dst, map, kb + 64 * b, row0,
                                                          tensor_z(q, tensor), bar);
                              else
-                                 ptx::tma_load_3d(dst, map, kb + b * bw, row0, tensor_z(q, tensor),
+                                 ptx::tma_load_3d(dst, map, kb + 64 * b, row0, tensor_z(q, tensor),
                                                   bar, pol_in);
                          });
         } else {
@@ -581,12 +688,13 @@ __device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& 
                          });
         }
     } else if (t < nthr) {
-        const int w0 = kb + 32 * (t >> 5);  // first position of this warp
-        const bool border = (w0 <= 0) || (w0 + 31 >= K - 1);
+        const int w0 = kb + 64 * (t >> 5);  // first position of this warp
+        const bool border = (w0 <= 0) || (w0 + 63 >= K - 1);
+        const bool local = p.g > 0 && p.g < L;
         if (border)
-            chain_consume<T, kRefine, VERT, FWD, true>(p, sm, ph, q, rank, pol_acc);
+            consume_dispatch<T, kRefine, VERT, FWD, true>(p, sm, ph, q, rank, pol_acc, local);
         else
-            chain_consume<T, kRefine, VERT, FWD, false>(p, sm, ph, q, rank, pol_acc);
+            consume_dispatch<T, kRefine, VERT, FWD, false>(p, sm, ph, q, rank, pol_acc, local);
     }
     __syncthreads();
 }
@@ -761,41 +869,38 @@ bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int W, int H, int64_
 
 int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
-// Geometry of one team size S; false if it does not fit.
+// Geometry of one team size S; false if it does not fit.  Owned ranges are
+// multiples of 64 positions (one vertical box per consumer warp).
 bool geometry_for(int S, int H, int W, int es, FusedPlan* gm) {
     FusedPlan g;
     memset(&g, 0, sizeof(g));
     g.S = S;
     g.T = S > 1 ? kHalo : 0;
+    const int seg = 32 / es;  // steps per stage
     if (S == 1) {
-        g.Kc_v = round_up(W, 8);
-        g.Kc_h = round_up(H, 8);
-        g.np_v = W;
-        g.np_h = H;
+        g.Kc_v = round_up(W, 64);
+        g.Kc_h = round_up(H, 64);
+        g.np_v = g.Kc_v;
+        g.np_h = g.Kc_h;
     } else {
-        g.Kc_v = round_up((W + S - 1) / S, 8);
-        g.Kc_h = round_up((H + S - 1) / S, 8);
-        if (g.Kc_v < g.T || g.Kc_h < g.T) return false;
+        g.Kc_v = round_up((W + S - 1) / S, 64);
+        g.Kc_h = round_up((H + S - 1) / S, 64);
+        // (on narrow planes the last CTAs may own no position of one
+        // orientation: they compute out-of-plane positions and exchange zeros)
         g.np_v = g.Kc_v + 2 * g.T;
         g.np_h = g.Kc_h + 2 * g.T;
     }
     const int npmax = g.np_v > g.np_h ? g.np_v : g.np_h;
-    const int tv = round_up(g.np_v, 32), th = round_up(g.np_h, 32);
-    g.threads = (tv > th ? tv : th) + 32;  // consumers + the producer warp
+    g.threads = npmax / 2 + 32;  // consumers (two positions each) + the producer warp
     if (g.threads > kMaxThreads) return false;
-    if (6 * ((g.np_v + 255) / 256) > 32 || 6 * ((g.np_h + 255) / 256) > 32) return false;
-    // horizontal tile: np_h rows x 32 bytes; box offsets 128-byte aligned (4 rows)
+    // vertical tile: np_v / 64 boxes of seg rows x 64 columns
+    g.nb_v = g.np_v / 64;
+    const int tile_v = g.nb_v * 64 * seg * es;
+    // horizontal tile: np_h rows x 32 bytes in boxes of <= 256 rows (multiple of 8)
     g.nb_h = (g.np_h + 255) / 256;
     g.bh_h = round_up((g.np_h + g.nb_h - 1) / g.nb_h, 8);
     if (g.bh_h > 256) return false;
     const int tile_h = g.nb_h * g.bh_h * 32;
-    // vertical tile: R rows x np_v columns in boxes of <= 256 columns (multiple of 8)
-    g.nb_v = (g.np_v + 255) / 256;
-    g.bw_v = round_up((g.np_v + g.nb_v - 1) / g.nb_v, 8);
-    if (g.bw_v > 256) return false;
-    g.R_v = 32 / es;  // one 32-byte row segment of steps, as horizontally
-    g.box_v = round_up(g.bw_v * g.R_v * es, 128);
-    const int tile_v = g.nb_v * g.box_v;
     g.tile_bytes = round_up(tile_h > tile_v ? tile_h : tile_v, 128);
     size_t a, b, c;
     g.stages = 0;
@@ -859,17 +964,17 @@ cudaError_t launch_typed(Problem& pb, const FusedPlan& fp, void* ws) {
     if (e != cudaSuccess) return e;
     const int H = (int)pb.H, W = (int)pb.W;
     const int nd = pb.d1 - pb.d0;
-    constexpr int J = 32 / (int)sizeof(T);  // horizontal box: 32-byte row segments
+    constexpr int J = 32 / (int)sizeof(T);  // steps per stage: 32-byte row segments
     FusedParams prm;
     memset(&prm, 0, sizeof(prm));
     const int64_t planes = pb.planes();
-    if (!encode_map(&prm.tm_xv, pb.x, pb.dtype, W, H, planes, fp.bw_v, fp.R_v) ||
+    if (!encode_map(&prm.tm_xv, pb.x, pb.dtype, W, H, planes, 64, J) ||
         !encode_map(&prm.tm_xh, pb.x, pb.dtype, W, H, planes, J, fp.bh_h))
         return cudaErrorInvalidValue;
     for (int d = pb.d0; d < pb.d1; ++d) {
         const bool vert = d < 2;
-        const int bx = vert ? fp.bw_v : J;
-        const int by = vert ? fp.R_v : fp.bh_h;
+        const int bx = vert ? 64 : J;
+        const int by = vert ? J : fp.bh_h;
         if (!encode_map(&prm.tm_z[d], pb.z.p[d], pb.dtype, W, H, 3 * planes, bx, by) ||
             !encode_map(&prm.tm_l[d], pb.lam.p[d], pb.dtype, W, H, planes, bx, by) ||
             !encode_map(&prm.tm_u[d], pb.u.p[d], pb.dtype, W, H, planes, bx, by))
@@ -893,14 +998,10 @@ cudaError_t launch_typed(Problem& pb, const FusedPlan& fp, void* ws) {
     prm.np_v = fp.np_v;
     prm.np_h = fp.np_h;
     prm.nb_v = fp.nb_v;
-    prm.bw_v = fp.bw_v;
-    prm.R_v = fp.R_v;
-    prm.box_v = fp.box_v;
     prm.nb_h = fp.nb_h;
     prm.bh_h = fp.bh_h;
     prm.tile_bytes = fp.tile_bytes;
     prm.stages = fp.stages;
-    prm.J_h = 32 / (int)sizeof(T);
     prm.n_slots = fp.n_slots;
     prm.n_items = (int)(planes * nd);
     prm.force_stale = fp.force_stale;
@@ -977,11 +1078,10 @@ cudaError_t launch_fused(Problem& pb, const FusedPlan& fp, void* ws, int* launch
     pb.kernel_name = "fused_kernel";
     if (getenv("GSPN_DEBUG_PLAN"))
         fprintf(stderr,
-                "gspn fused plan: S=%d T=%d Kc_v=%d Kc_h=%d np_v=%d np_h=%d nb_v=%d bw_v=%d R_v=%d "
-                "box_v=%d nb_h=%d bh_h=%d tile=%d stages=%d threads=%d smem=%zu teams=%d slots=%d\n",
-                fp.S, fp.T, fp.Kc_v, fp.Kc_h, fp.np_v, fp.np_h, fp.nb_v, fp.bw_v, fp.R_v, fp.box_v,
-                fp.nb_h, fp.bh_h, fp.tile_bytes, fp.stages, fp.threads, fp.smem, fp.n_teams,
-                fp.n_slots);
+                "gspn fused plan: S=%d T=%d Kc_v=%d Kc_h=%d np_v=%d np_h=%d nb_v=%d nb_h=%d "
+                "bh_h=%d tile=%d stages=%d threads=%d smem=%zu teams=%d slots=%d\n",
+                fp.S, fp.T, fp.Kc_v, fp.Kc_h, fp.np_v, fp.np_h, fp.nb_v, fp.nb_h, fp.bh_h,
+                fp.tile_bytes, fp.stages, fp.threads, fp.smem, fp.n_teams, fp.n_slots);
     cudaError_t e = pb.dtype == 0 ? launch_typed<float, true>(pb, fp, ws)
                                   : launch_typed<__nv_bfloat16, false>(pb, fp, ws);
     if (e == cudaSuccess) *launches += 1;

@@ -54,7 +54,7 @@ cudaError_t noalloc_scratch(int device, float** scratch);
 struct FusedPlan {
     int S, T;                 // CTAs per team (cluster), halo width
     int Kc_v, Kc_h, np_v, np_h;
-    int nb_v, bw_v, R_v, box_v, nb_h, bh_h;
+    int nb_v, nb_h, bh_h;
     int tile_bytes, threads, stages;
     size_t smem;
     int n_teams, n_slots;
