@@ -700,29 +700,42 @@ __device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& 
 }
 
 // Rounds the finished slot of plane q to the output dtype, writes y, re-zeroes
-// the slot.  CTA `rank` of the team takes a contiguous 1/S share.
+// the slot.  CTA `rank` of the team takes a contiguous 1/S share; every thread
+// keeps kUnroll 16-byte loads in flight so the pass runs at L2 bandwidth, not
+// at one load latency per thread.
 template <class T>
 __device__ __forceinline__ void convert_plane(const FusedParams& p, int q, int rank) {
+    constexpr int kUnroll = 8;
     const size_t HW = (size_t)p.H * p.W;
-    float* slot = p.slots + (size_t)(q % p.n_slots) * HW;
+    float4* slot = reinterpret_cast<float4*>(p.slots + (size_t)(q % p.n_slots) * HW);
     T* yq = static_cast<T*>(p.y) + (size_t)q * HW;
-    const size_t nvec = HW / 4;  // HW is a multiple of 4 (W * sizeof(T) % 16 == 0)
+    const size_t nvec = HW / 4;  // HW is a multiple of 4 (W * sizeof(T) % 32 == 0)
     const size_t per = (nvec + p.S - 1) / p.S;
     const size_t v0 = per * rank, v1 = min(nvec, v0 + per);
+    const size_t stride = blockDim.x;
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (size_t v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
-        float4* sp = reinterpret_cast<float4*>(slot) + v;
-        const float4 a = __ldcg(sp);
-        __stcg(sp, zero);
-        if constexpr (sizeof(T) == 4) {
-            __stcs(reinterpret_cast<float4*>(yq) + v, a);
-        } else {
-            __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(a.z, a.w);
-            uint2 packed;
-            packed.x = *reinterpret_cast<uint32_t*>(&lo);
-            packed.y = *reinterpret_cast<uint32_t*>(&hi);
-            __stcs(reinterpret_cast<uint2*>(yq) + v, packed);
+    for (size_t base = v0 + threadIdx.x; base < v1; base += kUnroll * stride) {
+        float4 a[kUnroll];
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+            const size_t v = base + j * stride;
+            if (v < v1) a[j] = __ldcg(slot + v);
+        }
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+            const size_t v = base + j * stride;
+            if (v >= v1) continue;
+            __stcg(slot + v, zero);
+            if constexpr (sizeof(T) == 4) {
+                __stcs(reinterpret_cast<float4*>(yq) + v, a[j]);
+            } else {
+                __nv_bfloat162 lo = __floats2bfloat162_rn(a[j].x, a[j].y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(a[j].z, a[j].w);
+                uint2 packed;
+                packed.x = *reinterpret_cast<uint32_t*>(&lo);
+                packed.y = *reinterpret_cast<uint32_t*>(&hi);
+                __stcs(reinterpret_cast<uint2*>(yq) + v, packed);
+            }
         }
     }
 }
