@@ -182,6 +182,26 @@ __device__ __forceinline__ void wait_bar(const FusedParams& p, Phases& ph, uint6
     }
 }
 
+// What a chain's consumer loop needs from the launch parameters and the
+// shared-memory carve-up, as plain values.  The consumer copies them once so
+// that no parameter is re-read after each shared-memory access.
+struct ChainEnv {
+    uint32_t full_s, empty_s, halo_s, rx_s;  // shared addresses of the barriers and halo buffer
+    unsigned long long timeout_ns;
+    FusedCtrl* ctrl;
+    int S;
+};
+
+__device__ __forceinline__ void wait_env(const ChainEnv& env, Phases& ph, uint32_t bar,
+                                         uint32_t parity, int code) {
+    if (ph.abort) return;
+    if (!ptx::wait_parity_bounded(bar, parity, env.timeout_ns)) {
+        ph.abort = true;
+        atomicCAS(&env.ctrl->call_error, 0, code);
+        atomicCAS(&env.ctrl->sticky_error, 0, code);
+    }
+}
+
 // Element e of a 16-byte vector of bf16 (e < 8) or fp32 (e < 4); e folds to a
 // constant inside fully unrolled loops.
 template <class T>
@@ -209,6 +229,14 @@ __device__ __forceinline__ void arm_halo_block(const FusedParams& p, const SmemV
     }
 }
 
+__device__ __forceinline__ void arm_halo_env(const ChainEnv& env, int rank, int blk, int L) {
+    if ((blk + 1) * kHalo < L) {
+        const uint32_t bytes =
+            sizeof(float) * kHalo * ((rank > 0 ? 1 : 0) + (rank < env.S - 1 ? 1 : 0));
+        ptx::mbar_arrive_expect_tx(env.halo_s + 8u * (blk & 1), bytes);
+    }
+}
+
 // First step > 0 at which a local group restarts (INT_MAX if none); later
 // restarts follow every g steps.
 __device__ __forceinline__ int first_restart(int g, int L, bool fwd) {
@@ -217,24 +245,32 @@ __device__ __forceinline__ int first_restart(int g, int L, bool fwd) {
 }
 
 // ------------------------------------------------------------------ pair math
-// A consumer thread owns two adjacent positions (k, k+1) of the line; their
-// values travel as packed fp32 pairs (position k in the low half).  A step's
-// weights are computed in two pipelined halves so the dependent chain between
-// two step barriers stays short:
-//   begin:    a_o = 2^-32 (1 + exp(-z_o)) for the three neighbours, lambda*x, u
-//   complete: p_o = product of the other two a's (0 for a missing neighbour),
-//             r = 1 / (p_0 + p_1 + p_2)
+// A consumer thread owns two positions of the line; their values travel as
+// packed fp32 pairs.  A step's weights are computed in two pipelined halves,
+// each in a different barrier interval, so that no instruction of an interval
+// waits for an exponential or a reciprocal issued in the same interval:
+//   begin:    e_o = 2^-32 exp(-z_o) for the three neighbours, lambda*x, u
+//   complete: a_o = e_o + 2^-32, p_o = product of the other two a's (0 for a
+//             missing neighbour), r = 1 / (p_0 + p_1 + p_2)
 // so that h = (p_0 h_left + p_1 h_self + p_2 h_right) r + lambda*x.
 struct PairA {
-    f2 a0, a1, a2, lx, u;
+    f2 e0, e1, e2, lx, u;  // exp(-z_o) * 2^-32 (0 for a missing neighbour), lambda*x, u
 };
 struct PairW {
     f2 p0, p1, p2, r, lx, u;
 };
-// Which neighbours exist (only consulted in warps that touch a border).
-struct PairFlags {
-    bool lo0, hi0, lo1, hi1;  // position k: k-1, k+1 exist; position k+1: k, k+2 exist
-    bool in0, in1;            // the positions lie inside the plane
+// Border handling without branches.  A neighbour outside the plane is
+// dropped: its a is the neutral scaled 1 and its product is 0.  Per thread
+// and half, m_lo / m_hi are 1 where the neighbour at offset -1 / +1 exists and
+// 0 where it does not; the exponent of a missing neighbour is forced to -inf
+// (ex2 gives 0, so a = 2^-32 exactly and no overflow can reach the masks).
+// Positions outside the plane need no forcing: their inputs are the zeros
+// the tensor maps fill in, their neighbours give them zero weight, and their
+// results are never accumulated.
+struct PairMask {
+    f2 m_lo, m_hi;        // 1 / 0
+    f2 kl_lo, ko_lo;      // exponent coefficients of slot 0: (-log2 e, -32) or (0, -inf)
+    f2 kl_hi, ko_hi;      // ... of slot 2
 };
 
 constexpr float kScale = 2.3283064365386963e-10f;  // 2^-32
@@ -256,10 +292,21 @@ __device__ __forceinline__ f2 ex2_pair(f2 t) {
     ptx::upk(t, a, b);
     return ptx::pk(ex2_approx(a), ex2_approx(b));
 }
-__device__ __forceinline__ f2 sel_pair(f2 v, bool keep0, bool keep1, float other) {
-    float a, b;
-    ptx::upk(v, a, b);
-    return ptx::pk(keep0 ? a : other, keep1 ? b : other);
+
+__device__ __forceinline__ PairMask make_mask(bool lo0, bool lo1, bool hi0, bool hi1) {
+    const float ninf = __int_as_float(0xff800000);
+    PairMask m;
+    m.m_lo = ptx::pk(lo0 ? 1.0f : 0.0f, lo1 ? 1.0f : 0.0f);
+    m.m_hi = ptx::pk(hi0 ? 1.0f : 0.0f, hi1 ? 1.0f : 0.0f);
+    m.kl_lo = ptx::pk(lo0 ? kNegLog2e : 0.0f, lo1 ? kNegLog2e : 0.0f);
+    m.ko_lo = ptx::pk(lo0 ? -32.0f : ninf, lo1 ? -32.0f : ninf);
+    m.kl_hi = ptx::pk(hi0 ? kNegLog2e : 0.0f, hi1 ? kNegLog2e : 0.0f);
+    m.ko_hi = ptx::pk(hi0 ? -32.0f : ninf, hi1 ? -32.0f : ninf);
+    return m;
+}
+
+__device__ __forceinline__ f2 bf16x2_pair(uint32_t w) {
+    return ptx::pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
 // The six inputs of one step for this thread's pair.
@@ -267,34 +314,53 @@ struct PairIn {
     f2 x, z0, z1, z2, lam, u;
 };
 
-template <bool kBorder>
-__device__ __forceinline__ PairA begin_pair(const PairIn& in, const PairFlags& f) {
-    const f2 kL = splat(kNegLog2e), kO = splat(-32.0f), kS = splat(kScale);
+// The six inputs as loaded from a vertical tile: one 32-bit word (two bf16)
+// or two floats per tensor; unpacked only when they are used.
+template <class T>
+struct RawIn {
+    typename std::conditional<sizeof(T) == 4, uint2, uint32_t>::type v[6];
+};
+template <class T>
+__device__ __forceinline__ PairIn unpack_raw(const RawIn<T>& r) {
+    f2 q[6];
+#pragma unroll
+    for (int k6 = 0; k6 < 6; ++k6) {
+        if constexpr (sizeof(T) == 4)
+            q[k6] = ptx::pk(__uint_as_float(r.v[k6].x), __uint_as_float(r.v[k6].y));
+        else
+            q[k6] = bf16x2_pair(r.v[k6]);
+    }
+    PairIn in;
+    in.x = q[0];
+    in.z0 = q[1];
+    in.z1 = q[2];
+    in.z2 = q[3];
+    in.lam = q[4];
+    in.u = q[5];
+    return in;
+}
+
+__device__ __forceinline__ PairA begin_pair(const PairIn& in, const PairMask& m) {
+    const f2 kL = splat(kNegLog2e), kO = splat(-32.0f);
     PairA A;
     A.lx = ptx::mul2(in.lam, in.x);
     A.u = in.u;
-    A.a0 = ptx::add2(ex2_pair(ptx::fma2(in.z0, kL, kO)), kS);
-    A.a1 = ptx::add2(ex2_pair(ptx::fma2(in.z1, kL, kO)), kS);
-    A.a2 = ptx::add2(ex2_pair(ptx::fma2(in.z2, kL, kO)), kS);
-    if (kBorder) {  // a missing neighbour: a = scaled 1 (neutral)
-        A.a0 = sel_pair(A.a0, f.lo0, f.lo1, kScale);
-        A.a2 = sel_pair(A.a2, f.hi0, f.hi1, kScale);
-    }
+    A.e0 = ex2_pair(ptx::fma2(in.z0, m.kl_lo, m.ko_lo));
+    A.e1 = ex2_pair(ptx::fma2(in.z1, kL, kO));
+    A.e2 = ex2_pair(ptx::fma2(in.z2, m.kl_hi, m.ko_hi));
     return A;
 }
 
-template <bool kRefine, bool kBorder>
-__device__ __forceinline__ PairW complete_pair(const PairA& A, const PairFlags& f) {
+template <bool kRefine>
+__device__ __forceinline__ PairW complete_pair(const PairA& A, const PairMask& m) {
+    const f2 kS = splat(kScale);
+    const f2 a0 = ptx::add2(A.e0, kS), a1 = ptx::add2(A.e1, kS), a2 = ptx::add2(A.e2, kS);
     PairW W;
     W.lx = A.lx;
     W.u = A.u;
-    W.p0 = ptx::mul2(A.a1, A.a2);
-    W.p1 = ptx::mul2(A.a0, A.a2);
-    W.p2 = ptx::mul2(A.a0, A.a1);
-    if (kBorder) {  // ... and product p = 0
-        W.p0 = sel_pair(W.p0, f.lo0, f.lo1, 0.0f);
-        W.p2 = sel_pair(W.p2, f.hi0, f.hi1, 0.0f);
-    }
+    W.p0 = ptx::mul2(ptx::mul2(a1, a2), m.m_lo);
+    W.p1 = ptx::mul2(a0, a2);
+    W.p2 = ptx::mul2(ptx::mul2(a0, a1), m.m_hi);
     const f2 sum = ptx::add2(ptx::add2(W.p0, W.p1), W.p2);
     float s0, s1;
     ptx::upk(sum, s0, s1);
@@ -306,50 +372,74 @@ __device__ __forceinline__ PairW complete_pair(const PairA& A, const PairFlags& 
     return W;
 }
 
-// h of the pair from the left neighbour pair (positions k-2, k-1), the pair's
-// own previous state and the right neighbour pair (k+2, k+3).
-__device__ __forceinline__ f2 finish_pair(const PairW& W, float left, f2 hs, float right) {
-    const f2 hl = ptx::pk(left, lo_of(hs));
-    const f2 hr = ptx::pk(hi_of(hs), right);
+// h of the pair from the previous states of the left neighbours (hl), the
+// positions themselves (hs) and the right neighbours (hr).
+__device__ __forceinline__ f2 finish_pair(const PairW& W, f2 hl, f2 hs, f2 hr) {
     return ptx::fma2(ptx::fma2(W.p2, hr, ptx::fma2(W.p1, hs, ptx::mul2(W.p0, hl))), W.r, W.lx);
 }
 
-__device__ __forceinline__ f2 bf16x2_pair(uint32_t w) {
-    return ptx::pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
 
 // Halo exchange after the last step of block blk.  Senders push their exact
 // pair to a neighbour CTA; halo threads return the received pair (others
 // return h unchanged).  Window position of this thread's pair: 2 * threadIdx.x.
-__device__ __forceinline__ f2 halo_exchange(const FusedParams& p, const SmemView& sm, Phases& ph,
-                                            int rank, int Kc, int blk, int L, f2 h) {
+__device__ __forceinline__ f2 halo_exchange(const ChainEnv& env, Phases& ph, int rank, int Kc,
+                                            int blk, int L, f2 h) {
     const int t = threadIdx.x;
     const int pos = 2 * t;
     const int par = blk & 1;
+    const uint32_t rx_side0 = env.rx_s + 4u * (par * 2 + 0) * kHalo;  // left halo of a CTA
+    const uint32_t rx_side1 = env.rx_s + 4u * (par * 2 + 1) * kHalo;  // right halo of a CTA
+    const uint32_t bar = env.halo_s + 8u * par;
     float a, b;
     ptx::upk(h, a, b);
-    if (rank > 0 && pos >= kHalo && pos < 2 * kHalo) {  // first owned -> left neighbour's right halo
-        const uint32_t ra =
-            ptx::map_shared(ptx::smem_addr(sm.rx + (par * 2 + 1) * kHalo + (pos - kHalo)), rank - 1);
-        const uint32_t rb = ptx::map_shared(ptx::smem_addr(sm.halo_bar + par), rank - 1);
-        ptx::st_async_f32x2(ra, a, b, rb);
-    }
-    if (rank < p.S - 1 && pos >= Kc && pos < Kc + kHalo) {  // last owned -> right neighbour's left halo
-        const uint32_t ra =
-            ptx::map_shared(ptx::smem_addr(sm.rx + (par * 2 + 0) * kHalo + (pos - Kc)), rank + 1);
-        const uint32_t rb = ptx::map_shared(ptx::smem_addr(sm.halo_bar + par), rank + 1);
-        ptx::st_async_f32x2(ra, a, b, rb);
-    }
+    if (rank > 0 && pos >= kHalo && pos < 2 * kHalo)  // first owned -> left neighbour's right halo
+        ptx::st_async_f32x2(ptx::map_shared(rx_side1 + 4u * (pos - kHalo), rank - 1), a, b,
+                            ptx::map_shared(bar, rank - 1));
+    if (rank < env.S - 1 && pos >= Kc && pos < Kc + kHalo)  // last owned -> right neighbour's left halo
+        ptx::st_async_f32x2(ptx::map_shared(rx_side0 + 4u * (pos - Kc), rank + 1), a, b,
+                            ptx::map_shared(bar, rank + 1));
     const bool recv_l = rank > 0 && pos < kHalo;
-    const bool recv_r = rank < p.S - 1 && pos >= kHalo + Kc && pos < 2 * kHalo + Kc;
+    const bool recv_r = rank < env.S - 1 && pos >= kHalo + Kc && pos < 2 * kHalo + Kc;
     if (recv_l || recv_r || t == 0) {
-        wait_bar(p, ph, sm.halo_bar + par, (ph.halo >> par) & 1u, 3);
+        wait_env(env, ph, bar, (ph.halo >> par) & 1u, 3);
         uint2 v = make_uint2(0u, 0u);
-        if (recv_l) v = ptx::lds_v2(ptx::smem_addr(sm.rx + (par * 2 + 0) * kHalo + pos));
-        if (recv_r) v = ptx::lds_v2(ptx::smem_addr(sm.rx + (par * 2 + 1) * kHalo + (pos - kHalo - Kc)));
+        if (recv_l) v = ptx::lds_v2(rx_side0 + 4u * pos);
+        if (recv_r) v = ptx::lds_v2(rx_side1 + 4u * (pos - kHalo - Kc));
         if (recv_l || recv_r) h = ptx::pk(__uint_as_float(v.x), __uint_as_float(v.y));
     }
-    if (t == 0) arm_halo_block(p, sm, rank, blk + 2, L);
+    if (t == 0) arm_halo_env(env, rank, blk + 2, L);
+    ph.halo ^= 1u << par;
+    return h;
+}
+
+// The same exchange for the horizontal thread mapping, where window position p
+// is half p / nthr of thread p % nthr: the owned edges and the halos are whole
+// low or high halves, so every sender or receiver moves one float.
+__device__ __forceinline__ f2 halo_exchange_split(const ChainEnv& env, Phases& ph, int rank,
+                                                  int Kc, int nthr, int blk, int L, f2 h) {
+    const int t = threadIdx.x;
+    const int par = blk & 1;
+    const uint32_t rx_side0 = env.rx_s + 4u * (par * 2 + 0) * kHalo;  // left halo of a CTA
+    const uint32_t rx_side1 = env.rx_s + 4u * (par * 2 + 1) * kHalo;  // right halo of a CTA
+    const uint32_t bar = env.halo_s + 8u * par;
+    float a, b;
+    ptx::upk(h, a, b);
+    const int pa = t, pb = t + nthr;  // window positions of the low and high halves
+    if (rank > 0 && pa >= kHalo && pa < 2 * kHalo)  // first owned -> left neighbour's right halo
+        ptx::st_async_f32(ptx::map_shared(rx_side1 + 4u * (pa - kHalo), rank - 1), a,
+                          ptx::map_shared(bar, rank - 1));
+    if (rank < env.S - 1 && pb >= Kc && pb < Kc + kHalo)  // last owned -> right neighbour's left halo
+        ptx::st_async_f32(ptx::map_shared(rx_side0 + 4u * (pb - Kc), rank + 1), b,
+                          ptx::map_shared(bar, rank + 1));
+    const bool recv_l = rank > 0 && pa < kHalo;
+    const bool recv_r = rank < env.S - 1 && pb >= kHalo + Kc && pb < 2 * kHalo + Kc;
+    if (recv_l || recv_r || t == 0) {
+        wait_env(env, ph, bar, (ph.halo >> par) & 1u, 3);
+        if (recv_l) a = ptx::lds_f32(rx_side0 + 4u * pa);
+        if (recv_r) b = ptx::lds_f32(rx_side1 + 4u * (pb - kHalo - Kc));
+        h = ptx::pk(a, b);
+    }
+    if (t == 0) arm_halo_env(env, rank, blk + 2, L);
     ph.halo ^= 1u << par;
     return h;
 }
@@ -390,12 +480,6 @@ __device__ __forceinline__ void producer_run(const FusedParams& p, const SmemVie
     }
 }
 
-// Consumer side: thread 0 releases slot `sl` after a barrier that follows the
-// consumers' last read of it.
-__device__ __forceinline__ void release_slot(const SmemView& sm, int sl) {
-    if (threadIdx.x == 0) ptx::mbar_arrive(ptx::smem_addr(sm.empty_bar + sl));
-}
-
 __device__ __forceinline__ const CUtensorMap* tensor_map(const FusedParams& p,
                                                          const CUtensorMap* xmap, int d,
                                                          int tensor) {
@@ -416,11 +500,17 @@ __device__ __forceinline__ int tensor_z(int q, int tensor) {
 // need W to be a multiple of kSeg (every stage full); a vertical chain's last
 // stage may run past the plane on zero-filled rows, whose results are not
 // accumulated.
-// Not inlined: each of the sixteen variants gets its own register allocation
-// (inlined together into the kernel they would share one and spill).
-template <class T, bool kRefine, bool VERT, bool FWD, bool kBorder, bool kLocal>
-__device__ __noinline__ Phases chain_consume(const FusedParams& p, const SmemView sm, Phases ph,
-                                             int q, int rank, uint64_t pol_acc) {
+template <class T, bool kRefine, bool VERT, bool FWD>
+__device__ __forceinline__ Phases chain_consume(const FusedParams& p, const SmemView& sm, Phases ph,
+                                                int q, int rank, uint64_t pol_acc) {
+    ChainEnv env;
+    env.full_s = ptx::smem_addr(sm.full_bar);
+    env.empty_s = ptx::smem_addr(sm.empty_bar);
+    env.halo_s = ptx::smem_addr(sm.halo_bar);
+    env.rx_s = ptx::smem_addr(sm.rx);
+    env.timeout_ns = p.timeout_ns;
+    env.ctrl = p.ctrl;
+    env.S = p.S;
     constexpr int kSeg = 32 / sizeof(T);
     constexpr int kPer = kSeg / 2;                   // steps per 16-byte half segment
     constexpr uint32_t kRowB = 64u * sizeof(T);      // vertical box row pitch
@@ -435,52 +525,74 @@ __device__ __noinline__ Phases chain_consume(const FusedParams& p, const SmemVie
     const int stages = p.stages, g_len = p.g;
     const bool multi = p.S > 1;
 
-    const int k = kb + 2 * t;
-    const bool own = k >= k0 && k < k0 + Kc && k < K;
-    const bool own1 = own && k + 1 < K;  // differs from own only at an odd K (horizontal)
-    PairFlags fl;
-    fl.lo0 = k > 0;
-    fl.hi0 = k + 1 < K;
-    fl.lo1 = k >= 0;
-    fl.hi1 = k + 2 < K;
-    fl.in0 = k >= 0 && k < K;
-    fl.in1 = k >= 0 && k + 1 < K;
+    // This thread's two positions: vertical k, k+1 (adjacent columns);
+    // horizontal k, k + nthr (rows in the two halves of the window), so that a
+    // warp's rows are consecutive and its neighbour pairs are the adjacent
+    // entries of the line buffer.
+    const int kA = VERT ? kb + 2 * t : kb + t;
+    const int kB = VERT ? kA + 1 : kA + nthr;
+    const bool ownA = kA >= k0 && kA < k0 + Kc && kA < K;
+    const bool ownB = kB >= k0 && kB < k0 + Kc && kB < K;
+    const PairMask fl = make_mask(kA != 0, kB != 0, kA != K - 1, kB != K - 1);
 
     const uint32_t ring_s = ptx::smem_addr(sm.ring);
     const uint32_t tb = p.tile_bytes;
-    const uint32_t col_byte = VERT ? warp * kBoxB + lane * (2u * (uint32_t)sizeof(T)) : 64u * t;
-    // line buffers: this pair at index 2t+2; neighbours pairs at 2t and 2t+4
-    const uint32_t hb0 = ptx::smem_addr(sm.hb) + 8u * t;
-    const uint32_t hb1 = hb0 + sm.line * 4;
+    // vertical: the pair's bytes in its warp's 64-column box; horizontal: row
+    // t of the row tile (32-byte rows, 16-byte halves swapped on every other
+    // group of four rows by the map's 32-byte swizzle); row t + nthr follows
+    // at 32 * nthr bytes with the same swizzle phase (nthr % 32 == 0)
+    const uint32_t col_byte = VERT ? warp * kBoxB + lane * (2u * (uint32_t)sizeof(T)) : 32u * t;
+    const uint32_t swz = VERT ? 0u : (uint32_t)((t >> 2) & 1);
+    // line buffers: 8-byte entry e at byte 8 (e + 1); this thread's entry is
+    // e = t, its neighbours e = t - 1 and t + 1 (vertical: the floats of the
+    // adjacent pairs; horizontal: whole entries)
+    const uint32_t hb_line0 = ptx::smem_addr(sm.hb);
+    const uint32_t hb_line1 = hb_line0 + sm.line * 4;
+    const uint32_t hb0 = hb_line0 + 8u * t;
+    const uint32_t hb1 = hb_line1 + 8u * t;
     float* const slot = p.slots + (size_t)(q % p.n_slots) * H * W;
-    float* const out_row = slot + (size_t)(own ? k : 0) * W;                   // horizontal
-    float* out_px = slot + (FWD ? 0 : (size_t)(H - 1) * W) + (own ? k : 0);  // vertical
+    float* const out_rowA = slot + (size_t)(ownA ? kA : 0) * W;                  // horizontal
+    float* const out_rowB = slot + (size_t)(ownB ? kB : 0) * W;
+    float* out_px = slot + (FWD ? 0 : (size_t)(H - 1) * W) + (ownA ? kA : 0);  // vertical
     const ptrdiff_t out_step = FWD ? W : -W;
 
-    uint4 v0[6], v1[6];  // horizontal: the current 16-byte half segment of rows k, k+1
+    uint4 v0[6], v1[6];  // horizontal: the current 16-byte half segment of rows kA, kB
     float acc0[4], acc1[4];
     int lsl = 0;         // slot of the next stage to acquire
     int rel_sl = 0;      // slot of the next stage to release
     int released = 0;
     auto acquire = [&]() {
-        wait_bar(p, ph, sm.full_bar + lsl, (ph.full >> lsl) & 1u, 1);
+        wait_env(env, ph, env.full_s + 8u * lsl, (ph.full >> lsl) & 1u, 1);
         ph.full ^= 1u << lsl;
         lsl = (lsl + 1 == stages) ? 0 : lsl + 1;
     };
     auto release = [&]() {
-        release_slot(sm, rel_sl);
+        if (t == 0) ptx::mbar_arrive(env.empty_s + 8u * rel_sl);
         rel_sl = (rel_sl + 1 == stages) ? 0 : rel_sl + 1;
         ++released;
     };
     auto tile_base = [&](int sl) -> uint32_t { return ring_s + sl * 6 * tb + col_byte; };
     // horizontal: load logical half jl (steps jl*kPer ..) of the stage in slot sl
     auto load_half = [&](int sl, int jl) {
-        const uint32_t b = tile_base(sl) + 16u * (FWD ? jl : 1 - jl);
+        const uint32_t b = tile_base(sl) + 16u * ((uint32_t)(FWD ? jl : 1 - jl) ^ swz);
 #pragma unroll
         for (int k6 = 0; k6 < 6; ++k6) {
             v0[k6] = ptx::lds_v4(b + k6 * tb);
-            v1[k6] = ptx::lds_v4(b + k6 * tb + 32u);
+            v1[k6] = ptx::lds_v4(b + k6 * tb + 32u * nthr);
         }
+    };
+    // vertical: raw inputs of step w of the stage in slot sl
+    auto fetch_raw = [&](int sl, int w) -> RawIn<T> {
+        RawIn<T> r;
+        const uint32_t b = tile_base(sl) + (FWD ? w : kSeg - 1 - w) * kRowB;
+#pragma unroll
+        for (int k6 = 0; k6 < 6; ++k6) {
+            if constexpr (sizeof(T) == 4)
+                r.v[k6] = ptx::lds_v2(b + k6 * tb);
+            else
+                r.v[k6] = ptx::lds_u32(b + k6 * tb);
+        }
+        return r;
     };
     // inputs of step w (0 <= w < kSeg) of the stage in slot sl
     auto fetch = [&](int sl, int w) -> PairIn {
@@ -511,13 +623,22 @@ __device__ __noinline__ Phases chain_consume(const FusedParams& p, const SmemVie
         return in;
     };
 
-    // Software pipeline: Wt = weights of the step about to run, A = first half
-    // of the next step's.
+    // Software pipeline.  In the barrier interval of step w a thread
+    //   issues the loads of the neighbour state of step w (the critical path)
+    //   and, vertically, the inputs of step w + 3;
+    //   completes the weights of step w + 1 and begins those of step w + 2
+    //   (inputs loaded one interval earlier), which covers the load latency;
+    //   finishes step w, stores its state and accumulates u * h.
+    // Vertical stage reads end at step kSeg - 4 (inputs of row kSeg - 1), so
+    // the stage is released after the barrier of step kSeg - 3; horizontal
+    // stages are copied to registers, the second half at step kPer - 2.
     int cur_sl = 0;
     acquire();
     if constexpr (!VERT) load_half(cur_sl, 0);
-    PairW Wt = complete_pair<kRefine, kBorder>(begin_pair<kBorder>(fetch(cur_sl, 0), fl), fl);
-    PairA A = begin_pair<kBorder>(fetch(cur_sl, 1), fl);
+    PairW Wt = complete_pair<kRefine>(begin_pair(fetch(cur_sl, 0), fl), fl);
+    PairA A = begin_pair(fetch(cur_sl, 1), fl);
+    RawIn<T> raw2;  // vertical: inputs of step w + 2
+    if constexpr (VERT) raw2 = fetch_raw(cur_sl, 2);
     f2 h = splat(0.0f);
     int next_rs = first_restart(g_len, L, FWD);
     for (int st = 0; st < nst; ++st) {
@@ -528,54 +649,76 @@ __device__ __noinline__ Phases chain_consume(const FusedParams& p, const SmemVie
             constexpr int w = decltype(wc)::value;
             bool start = false;
             if constexpr (w == 0) start = (st == 0);
-            if constexpr (kLocal) {
-                if (st * kSeg + w == next_rs) {
-                    start = true;
-                    next_rs += g_len;
-                }
+            if (st * kSeg + w == next_rs) {  // local groups (never true for a global scan)
+                start = true;
+                next_rs += g_len;
             }
             if (w > 0 || st > 0) {
                 ptx::named_barrier(1, nthr);
-                // the barrier follows the last read of the current stage:
-                // vertical fetches row kSeg-1 at step kSeg-3, horizontal loads
-                // its second half at step kPer-2
-                if constexpr (w == (VERT ? kSeg - 2 : kPer - 1)) release();
+                if constexpr (w == (VERT ? kSeg - 3 : kPer - 1)) release();
             }
             const uint32_t hprev = (w & 1) ? hb0 : hb1;
             const uint32_t hcur = (w & 1) ? hb1 : hb0;
-            // 1. neighbour state (the critical path)
+            // 1. neighbour state of step w
             const uint2 lp = ptx::lds_v2(hprev);
             const uint2 rp = ptx::lds_v2(hprev + 16u);
-            // 2. shared-memory inputs of step w + 2 (vertical: six loads;
-            //    horizontal: the next half segment when step w + 2 starts one)
-            constexpr bool kNext = w + 2 >= kSeg;     // step w + 2 is in the next stage
-            constexpr int w2 = kNext ? w + 2 - kSeg : w + 2;
-            const bool have2 = !kNext || more;
-            const int sl2 = kNext ? nxt_sl : cur_sl;
-            if constexpr (kNext && w2 == 0) {
-                if (more) {
-                    acquire();
-                    if constexpr (!VERT) load_half(nxt_sl, 0);
-                }
-            }
-            if constexpr (!VERT && !kNext && w2 == kPer) load_half(cur_sl, 1);
-            PairIn in2;
+            // 2. shared-memory inputs: vertical step w + 3; horizontal the half
+            //    segment that step w + 2 starts, if it starts one
+            constexpr bool kNext2 = w + 2 >= kSeg;  // step w + 2 is in the next stage
+            constexpr int w2 = kNext2 ? w + 2 - kSeg : w + 2;
+            const bool have2 = !kNext2 || more;
+            RawIn<T> raw3;
             if constexpr (VERT) {
-                if (have2) in2 = fetch(sl2, w2);
+                constexpr bool kNext3 = w + 3 >= kSeg;
+                constexpr int w3 = kNext3 ? w + 3 - kSeg : w + 3;
+                if constexpr (!kNext3) {
+                    raw3 = fetch_raw(cur_sl, w3);
+                } else {
+                    if (more) {
+                        if constexpr (w3 == 0) acquire();
+                        raw3 = fetch_raw(nxt_sl, w3);
+                    }
+                }
+            } else {
+                if constexpr (kNext2 && w2 == 0) {
+                    if (more) {
+                        acquire();
+                        load_half(nxt_sl, 0);
+                    }
+                }
+                if constexpr (!kNext2 && w2 == kPer) load_half(cur_sl, 1);
             }
-            // 3. this step's state
-            f2 hn = start ? Wt.lx
-                          : finish_pair(Wt, __uint_as_float(lp.y), h, __uint_as_float(rp.x));
-            if (kBorder) hn = sel_pair(hn, fl.in0, fl.in1, 0.0f);
-            h = hn;
+            // 3. weights of step w + 1 (registers) and first half of step w + 2's
+            const PairW Wn = complete_pair<kRefine>(A, fl);
+            if (have2) {
+                if constexpr (VERT)
+                    A = begin_pair(unpack_raw<T>(raw2), fl);
+                else
+                    A = begin_pair(fetch(kNext2 ? nxt_sl : cur_sl, w2), fl);
+            }
+            // 4. this step's state
+            f2 hl, hr;
+            if constexpr (VERT) {
+                hl = ptx::pk(__uint_as_float(lp.y), lo_of(h));
+                hr = ptx::pk(hi_of(h), __uint_as_float(rp.x));
+            } else {
+                hl = ptx::pk(__uint_as_float(lp.x), __uint_as_float(lp.y));
+                hr = ptx::pk(__uint_as_float(rp.x), __uint_as_float(rp.y));
+            }
+            h = start ? Wt.lx : finish_pair(Wt, hl, h, hr);
             {
                 float a, b;
                 ptx::upk(h, a, b);
                 ptx::sts_v2_f32(hcur + 8u, a, b);
+                if constexpr (!VERT) {  // the seam between the window's two halves
+                    const uint32_t line = (w & 1) ? hb_line1 : hb_line0;
+                    if (t == nthr - 1) ptx::sts_f32(line + 4u, a);               // left of kB(0)
+                    if (t == 0) ptx::sts_f32(line + 8u * (nthr + 1), b);       // right of kA(nthr-1)
+                }
             }
             const f2 uh = ptx::mul2(Wt.u, h);
             if constexpr (VERT) {
-                if (own && w < wlim) {
+                if (ownA && w < wlim) {
                     float a, b;
                     ptx::upk(uh, a, b);
                     ptx::red_add_v2_f32(out_px, a, b, pol_acc);
@@ -588,25 +731,23 @@ __device__ __noinline__ Phases chain_consume(const FusedParams& p, const SmemVie
                 acc1[FWD ? (w & 3) : 3 - (w & 3)] = b;
                 if constexpr ((w & 3) == 3) {
                     const int c0 = FWD ? st * kSeg + (w - 3) : W - st * kSeg - (w + 1);
-                    if (own)
-                        ptx::red_add_v4_f32_hint(out_row + c0, acc0[0], acc0[1], acc0[2], acc0[3],
+                    if (ownA)
+                        ptx::red_add_v4_f32_hint(out_rowA + c0, acc0[0], acc0[1], acc0[2], acc0[3],
                                                  pol_acc);
-                    if (own1)
-                        ptx::red_add_v4_f32_hint(out_row + W + c0, acc1[0], acc1[1], acc1[2],
+                    if (ownB)
+                        ptx::red_add_v4_f32_hint(out_rowB + c0, acc1[0], acc1[1], acc1[2],
                                                  acc1[3], pol_acc);
                 }
             }
-            // 4. weights of step w + 1, first half of step w + 2's
-            Wt = complete_pair<kRefine, kBorder>(A, fl);
-            if (have2) {
-                if constexpr (!VERT) in2 = fetch(sl2, w2);
-                A = begin_pair<kBorder>(in2, fl);
-            }
+            Wt = Wn;
+            if constexpr (VERT) raw2 = raw3;
         });
         cur_sl = nxt_sl;
         // halo exchange at the end of every 32-step block that has a successor
         if (multi && ((st + 1) * kSeg) % kHalo == 0 && (st + 1) * kSeg < L) {
-            const f2 hx = halo_exchange(p, sm, ph, rank, Kc, (st + 1) * kSeg / kHalo - 1, L, h);
+            const int blk = (st + 1) * kSeg / kHalo - 1;
+            const f2 hx = VERT ? halo_exchange(env, ph, rank, Kc, blk, L, h)
+                               : halo_exchange_split(env, ph, rank, Kc, nthr, blk, L, h);
             if (hx != h) {
                 h = hx;
                 float a, b;
@@ -635,16 +776,6 @@ __device__ __forceinline__ void chain_begin(const FusedParams& p, const SmemView
         arm_halo_block(p, sm, rank, 1, L);
     }
     __syncthreads();
-}
-
-template <class T, bool kRefine, bool VERT, bool FWD, bool kBorder>
-__device__ __forceinline__ void consume_dispatch(const FusedParams& p, const SmemView& sm,
-                                                 Phases& ph, int q, int rank, uint64_t pol_acc,
-                                                 bool local) {
-    if (local)
-        ph = chain_consume<T, kRefine, VERT, FWD, kBorder, true>(p, sm, ph, q, rank, pol_acc);
-    else
-        ph = chain_consume<T, kRefine, VERT, FWD, kBorder, false>(p, sm, ph, q, rank, pol_acc);
 }
 
 template <class T, bool kRefine, bool VERT, bool FWD>
@@ -688,13 +819,7 @@ __device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& 
                          });
         }
     } else if (t < nthr) {
-        const int w0 = kb + 64 * (t >> 5);  // first position of this warp
-        const bool border = (w0 <= 0) || (w0 + 63 >= K - 1);
-        const bool local = p.g > 0 && p.g < L;
-        if (border)
-            consume_dispatch<T, kRefine, VERT, FWD, true>(p, sm, ph, q, rank, pol_acc, local);
-        else
-            consume_dispatch<T, kRefine, VERT, FWD, false>(p, sm, ph, q, rank, pol_acc, local);
+        ph = chain_consume<T, kRefine, VERT, FWD>(p, sm, ph, q, rank, pol_acc);
     }
     __syncthreads();
 }
@@ -761,7 +886,9 @@ template <class T, bool kRefine>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     fused_kernel(const __grid_constant__ FusedParams p) {
     extern __shared__ __align__(128) char smem_raw[];
-    const SmemView sm = carve(smem_raw, p);
+    // TMA destinations sit on 1024-byte boundaries (the horizontal maps are swizzled)
+    char* const smem_base = smem_raw + ((1024u - (ptx::smem_addr(smem_raw) & 1023u)) & 1023u);
+    const SmemView sm = carve(smem_base, p);
     const int rank = p.S > 1 ? (int)ptx::cluster_ctarank() : 0;
     const int t = threadIdx.x;
 
@@ -865,7 +992,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int W, int H, int64_t depth, int box_x,
-                int box_y) {
+                int box_y, bool swizzle32 = false) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const size_t es = dtype == 0 ? 4 : 2;
@@ -875,7 +1002,8 @@ bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int W, int H, int64_
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                      3, const_cast<void*>(ptr), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     swizzle32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -911,14 +1039,14 @@ bool geometry_for(int S, int H, int W, int es, FusedPlan* gm) {
     const int tile_v = g.nb_v * 64 * seg * es;
     // horizontal tile: np_h rows x 32 bytes in boxes of <= 256 rows (multiple of 8)
     g.nb_h = (g.np_h + 255) / 256;
-    g.bh_h = round_up((g.np_h + g.nb_h - 1) / g.nb_h, 8);
+    g.bh_h = round_up((g.np_h + g.nb_h - 1) / g.nb_h, 32);  // boxes on 1024-byte boundaries
     if (g.bh_h > 256) return false;
     const int tile_h = g.nb_h * g.bh_h * 32;
-    g.tile_bytes = round_up(tile_h > tile_v ? tile_h : tile_v, 128);
+    g.tile_bytes = round_up(tile_h > tile_v ? tile_h : tile_v, 1024);
     size_t a, b, c;
     g.stages = 0;
     for (int st = kMaxStages; st >= 2; --st) {
-        g.smem = smem_layout(g.tile_bytes, st, npmax, &a, &b, &c);
+        g.smem = smem_layout(g.tile_bytes, st, npmax, &a, &b, &c) + 1024;  // + base alignment
         if (g.smem <= 227 * 1024) {
             g.stages = st;
             break;
@@ -982,15 +1110,15 @@ cudaError_t launch_typed(Problem& pb, const FusedPlan& fp, void* ws) {
     memset(&prm, 0, sizeof(prm));
     const int64_t planes = pb.planes();
     if (!encode_map(&prm.tm_xv, pb.x, pb.dtype, W, H, planes, 64, J) ||
-        !encode_map(&prm.tm_xh, pb.x, pb.dtype, W, H, planes, J, fp.bh_h))
+        !encode_map(&prm.tm_xh, pb.x, pb.dtype, W, H, planes, J, fp.bh_h, true))
         return cudaErrorInvalidValue;
     for (int d = pb.d0; d < pb.d1; ++d) {
         const bool vert = d < 2;
         const int bx = vert ? 64 : J;
         const int by = vert ? J : fp.bh_h;
-        if (!encode_map(&prm.tm_z[d], pb.z.p[d], pb.dtype, W, H, 3 * planes, bx, by) ||
-            !encode_map(&prm.tm_l[d], pb.lam.p[d], pb.dtype, W, H, planes, bx, by) ||
-            !encode_map(&prm.tm_u[d], pb.u.p[d], pb.dtype, W, H, planes, bx, by))
+        if (!encode_map(&prm.tm_z[d], pb.z.p[d], pb.dtype, W, H, 3 * planes, bx, by, !vert) ||
+            !encode_map(&prm.tm_l[d], pb.lam.p[d], pb.dtype, W, H, planes, bx, by, !vert) ||
+            !encode_map(&prm.tm_u[d], pb.u.p[d], pb.dtype, W, H, planes, bx, by, !vert))
             return cudaErrorInvalidValue;
     }
     char* base = static_cast<char*>(ws);
