@@ -1178,7 +1178,7 @@ bool fused_plan(const Problem& pb, FusedPlan* fp) {
     const int H = (int)pb.H, W = (int)pb.W;
     const int nd = pb.d1 - pb.d0;
     const size_t slot_bytes = sizeof(float) * (size_t)H * W;
-    const size_t l2_budget = (size_t)80 << 20;
+    const size_t l2_budget = (size_t)96 << 20;
     for (int S : {1, 2, 4, 8}) {
         FusedPlan plan;
         if (!geometry_for(S, H, W, es, &plan)) continue;
