@@ -541,7 +541,11 @@ __device__ __forceinline__ Phases chain_consume(const FusedParams& p, const Smem
     // t of the row tile (32-byte rows, 16-byte halves swapped on every other
     // group of four rows by the map's 32-byte swizzle); row t + nthr follows
     // at 32 * nthr bytes with the same swizzle phase (nthr % 32 == 0)
-    const uint32_t col_byte = VERT ? warp * kBoxB + lane * (2u * (uint32_t)sizeof(T)) : 32u * t;
+    // vertical: a stage holds, per warp, the six tensors' 64-column boxes
+    // back to back ([warp][tensor][row][64 columns]), so every input load of a
+    // step is this base plus a compile-time offset
+    const uint32_t col_byte =
+        VERT ? warp * (6u * kBoxB) + lane * (2u * (uint32_t)sizeof(T)) : 32u * t;
     const uint32_t swz = VERT ? 0u : (uint32_t)((t >> 2) & 1);
     // line buffers: 8-byte entry e at byte 8 (e + 1); this thread's entry is
     // e = t, its neighbours e = t - 1 and t + 1 (vertical: the floats of the
@@ -582,38 +586,26 @@ __device__ __forceinline__ Phases chain_consume(const FusedParams& p, const Smem
         }
     };
     // vertical: raw inputs of step w of the stage in slot sl
-    auto fetch_raw = [&](int sl, int w) -> RawIn<T> {
+    auto fetch_raw = [&](uint32_t base, int w) -> RawIn<T> {
         RawIn<T> r;
-        const uint32_t b = tile_base(sl) + (FWD ? w : kSeg - 1 - w) * kRowB;
+        const uint32_t b = base + (FWD ? w : kSeg - 1 - w) * kRowB;
 #pragma unroll
         for (int k6 = 0; k6 < 6; ++k6) {
             if constexpr (sizeof(T) == 4)
-                r.v[k6] = ptx::lds_v2(b + k6 * tb);
+                r.v[k6] = ptx::lds_v2(b + k6 * kBoxB);
             else
-                r.v[k6] = ptx::lds_u32(b + k6 * tb);
+                r.v[k6] = ptx::lds_u32(b + k6 * kBoxB);
         }
         return r;
     };
     // inputs of step w (0 <= w < kSeg) of the stage in slot sl
     auto fetch = [&](int sl, int w) -> PairIn {
+        if constexpr (VERT) return unpack_raw<T>(fetch_raw(tile_base(sl), w));
         PairIn in;
         f2 r[6];
-        if constexpr (VERT) {
-            const uint32_t b = tile_base(sl) + (FWD ? w : kSeg - 1 - w) * kRowB;
+        const int e = FWD ? (w % kPer) : (kPer - 1 - (w % kPer));
 #pragma unroll
-            for (int k6 = 0; k6 < 6; ++k6) {
-                if constexpr (sizeof(T) == 4) {
-                    const uint2 u2 = ptx::lds_v2(b + k6 * tb);
-                    r[k6] = ptx::pk(__uint_as_float(u2.x), __uint_as_float(u2.y));
-                } else {
-                    r[k6] = bf16x2_pair(ptx::lds_u32(b + k6 * tb));
-                }
-            }
-        } else {
-            const int e = FWD ? (w % kPer) : (kPer - 1 - (w % kPer));
-#pragma unroll
-            for (int k6 = 0; k6 < 6; ++k6) r[k6] = ptx::pk(vec_elem<T>(v0[k6], e), vec_elem<T>(v1[k6], e));
-        }
+        for (int k6 = 0; k6 < 6; ++k6) r[k6] = ptx::pk(vec_elem<T>(v0[k6], e), vec_elem<T>(v1[k6], e));
         in.x = r[0];
         in.z0 = r[1];
         in.z1 = r[2];
@@ -638,21 +630,24 @@ __device__ __forceinline__ Phases chain_consume(const FusedParams& p, const Smem
     PairW Wt = complete_pair<kRefine>(begin_pair(fetch(cur_sl, 0), fl), fl);
     PairA A = begin_pair(fetch(cur_sl, 1), fl);
     RawIn<T> raw2;  // vertical: inputs of step w + 2
-    if constexpr (VERT) raw2 = fetch_raw(cur_sl, 2);
+    if constexpr (VERT) raw2 = fetch_raw(tile_base(cur_sl), 2);
     f2 h = splat(0.0f);
     int next_rs = first_restart(g_len, L, FWD);
     for (int st = 0; st < nst; ++st) {
         const int nxt_sl = (cur_sl + 1 == stages) ? 0 : cur_sl + 1;
         const bool more = st + 1 < nst;
-        const int wlim = more ? kSeg : L - st * kSeg;  // vertical: steps inside the plane
+        // vertical: steps of this stage inside the plane (0 if not owned)
+        const int wl = !ownA ? 0 : more ? kSeg : L - st * kSeg;
+        const uint32_t cur_base = tile_base(cur_sl), nxt_base = tile_base(nxt_sl);
+        // steps of this stage that start a group (bit w)
+        uint32_t starts = st == 0 ? 1u : 0u;
+        while (next_rs < (st + 1) * kSeg) {
+            starts |= 1u << (next_rs - st * kSeg);
+            next_rs += g_len;
+        }
         static_for<kSeg>([&](auto wc) {
             constexpr int w = decltype(wc)::value;
-            bool start = false;
-            if constexpr (w == 0) start = (st == 0);
-            if (st * kSeg + w == next_rs) {  // local groups (never true for a global scan)
-                start = true;
-                next_rs += g_len;
-            }
+            const bool start = (starts >> w) & 1u;
             if (w > 0 || st > 0) {
                 ptx::named_barrier(1, nthr);
                 if constexpr (w == (VERT ? kSeg - 3 : kPer - 1)) release();
@@ -672,11 +667,11 @@ __device__ __forceinline__ Phases chain_consume(const FusedParams& p, const Smem
                 constexpr bool kNext3 = w + 3 >= kSeg;
                 constexpr int w3 = kNext3 ? w + 3 - kSeg : w + 3;
                 if constexpr (!kNext3) {
-                    raw3 = fetch_raw(cur_sl, w3);
+                    raw3 = fetch_raw(cur_base, w3);
                 } else {
                     if (more) {
                         if constexpr (w3 == 0) acquire();
-                        raw3 = fetch_raw(nxt_sl, w3);
+                        raw3 = fetch_raw(nxt_base, w3);
                     }
                 }
             } else {
@@ -705,23 +700,23 @@ __device__ __forceinline__ Phases chain_consume(const FusedParams& p, const Smem
                 hl = ptx::pk(__uint_as_float(lp.x), __uint_as_float(lp.y));
                 hr = ptx::pk(__uint_as_float(rp.x), __uint_as_float(rp.y));
             }
-            h = start ? Wt.lx : finish_pair(Wt, hl, h, hr);
+            h = ptx::sel64(start, Wt.lx, finish_pair(Wt, hl, h, hr));
             {
                 float a, b;
                 ptx::upk(h, a, b);
                 ptx::sts_v2_f32(hcur + 8u, a, b);
                 if constexpr (!VERT) {  // the seam between the window's two halves
                     const uint32_t line = (w & 1) ? hb_line1 : hb_line0;
-                    if (t == nthr - 1) ptx::sts_f32(line + 4u, a);               // left of kB(0)
-                    if (t == 0) ptx::sts_f32(line + 8u * (nthr + 1), b);       // right of kA(nthr-1)
+                    ptx::sts_f32_if(t == nthr - 1, line + 4u, a);           // left of kB(0)
+                    ptx::sts_f32_if(t == 0, line + 8u * (nthr + 1), b);   // right of kA(nthr-1)
                 }
             }
             const f2 uh = ptx::mul2(Wt.u, h);
             if constexpr (VERT) {
-                if (ownA && w < wlim) {
+                {
                     float a, b;
                     ptx::upk(uh, a, b);
-                    ptx::red_add_v2_f32(out_px, a, b, pol_acc);
+                    ptx::red_add_v2_f32_if(w < wl, out_px, a, b, pol_acc);
                 }
                 out_px += out_step;
             } else {
@@ -731,12 +726,10 @@ __device__ __forceinline__ Phases chain_consume(const FusedParams& p, const Smem
                 acc1[FWD ? (w & 3) : 3 - (w & 3)] = b;
                 if constexpr ((w & 3) == 3) {
                     const int c0 = FWD ? st * kSeg + (w - 3) : W - st * kSeg - (w + 1);
-                    if (ownA)
-                        ptx::red_add_v4_f32_hint(out_rowA + c0, acc0[0], acc0[1], acc0[2], acc0[3],
-                                                 pol_acc);
-                    if (ownB)
-                        ptx::red_add_v4_f32_hint(out_rowB + c0, acc1[0], acc1[1], acc1[2],
-                                                 acc1[3], pol_acc);
+                    ptx::red_add_v4_f32_if(ownA, out_rowA + c0, acc0[0], acc0[1], acc0[2], acc0[3],
+                                           pol_acc);
+                    ptx::red_add_v4_f32_if(ownB, out_rowB + c0, acc1[0], acc1[1], acc1[2], acc1[3],
+                                           pol_acc);
                 }
             }
             Wt = Wn;
@@ -798,8 +791,9 @@ __device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& 
             producer_run(p, sm, ps, nst, nb, 6u * nb * 64u * kSeg * sizeof(T),
                          [&](int st, int sl, int tensor, int b, uint32_t bar) {
                              const int row0 = FWD ? st * kSeg : H - kSeg - st * kSeg;
-                             const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) +
-                                                  b * (64u * kSeg * (uint32_t)sizeof(T));
+                             constexpr uint32_t kBox = 64u * kSeg * (uint32_t)sizeof(T);
+                             const uint32_t dst = ptx::smem_addr(sm.tile(sl, 0)) +
+                                                  (b * 6u + tensor) * kBox;
                              const CUtensorMap* map = tensor_map(p, &p.tm_xv, d, tensor);
                              if (tensor == 0)
                                  ptx::tma_load_3d_normal(dst, map, kb + 64 * b, row0,

@@ -156,6 +156,32 @@ __device__ __forceinline__ void red_add_v4_f32_hint(float* addr, float a, float 
         "f"(a), "f"(b), "f"(c), "f"(d), "l"(policy)
         : "memory");
 }
+// Predicated forms: the instruction is skipped (no branch) when `on` is 0.
+__device__ __forceinline__ void red_add_v2_f32_if(bool on, float* addr, float a, float b,
+                                                  uint64_t policy) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %0, 0;\n\t"
+        "@p red.relaxed.gpu.global.add.L2::cache_hint.v2.f32 [%1], {%2, %3}, %4;\n\t}" ::"r"(
+            (uint32_t)on),
+        "l"(addr), "f"(a), "f"(b), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ void red_add_v4_f32_if(bool on, float* addr, float a, float b, float c,
+                                                  float d, uint64_t policy) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %0, 0;\n\t"
+        "@p red.relaxed.gpu.global.add.L2::cache_hint.v4.f32 [%1], {%2, %3, %4, %5}, %6;\n\t}" ::"r"(
+            (uint32_t)on),
+        "l"(addr), "f"(a), "f"(b), "f"(c), "f"(d), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ void sts_f32_if(bool on, uint32_t a, float v) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %0, 0;\n\t@p st.shared.f32 [%1], %2;\n\t}" ::"r"(
+            (uint32_t)on),
+        "r"(a), "f"(v)
+        : "memory");
+}
 // Plain arrive (count 1) on a CTA-local mbarrier, release semantics.
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
@@ -232,6 +258,15 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
 }
 
 // ---- packed fp32 pairs (sm_100 f32x2 arithmetic) -------------------------------
+// a if c else b, without a branch.
+__device__ __forceinline__ unsigned long long sel64(bool c, unsigned long long a,
+                                                    unsigned long long b) {
+    unsigned long long r;
+    asm("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %3, 0;\n\tselp.b64 %0, %1, %2, p;\n\t}"
+        : "=l"(r)
+        : "l"(a), "l"(b), "r"((uint32_t)c));
+    return r;
+}
 // A pair holds position A in the low half and position B in the high half.
 typedef unsigned long long f2;
 __device__ __forceinline__ f2 pk(float a, float b) {
