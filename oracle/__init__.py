@@ -70,6 +70,9 @@ def _load():
             lib.gspn_oracle_forward.argtypes = [_dp, arr4, arr4, arr4, i64, i64, i64, i64, i64,
                                                 ctypes.c_int, _dp]
             lib.gspn_oracle_forward.restype = ctypes.c_int
+            lib.gspn_oracle_backward.argtypes = [_dp, arr4, arr4, arr4, _dp, i64, i64, i64, i64,
+                                                 i64, ctypes.c_int, _dp, arr4, arr4, arr4]
+            lib.gspn_oracle_backward.restype = ctypes.c_int
             lib.gspn_oracle_default_threads.argtypes = []
             lib.gspn_oracle_default_threads.restype = ctypes.c_int
             _lib = lib
@@ -137,3 +140,29 @@ def forward(x, wlogit, lam, u, group_len: int = 0, nthreads: int = 0) -> np.ndar
     if rc != 0:
         raise ValueError(f"oracle rejected arguments (rc={rc})")
     return y
+
+
+def backward(x, wlogit, lam, u, gy, group_len: int = 0, nthreads: int = 0):
+    """Gradients of L = sum(gy * y) in fp64 (chain rule on the forward
+    definition; the walkthrough's section "反向传播" describes the adjoint
+    flowing back from later lines).  Returns (dx, dwlogit[4], dlam[4], du[4])."""
+    x = as_f64(x)
+    gy = as_f64(gy)
+    B, C, H, W = x.shape
+    assert gy.shape == x.shape
+    zs = [as_f64(t) for t in wlogit]
+    ls = [as_f64(t) for t in lam]
+    us = [as_f64(t) for t in u]
+    dx = np.empty_like(x)
+    dz = [np.empty_like(z) for z in zs]
+    dl = [np.empty_like(x) for _ in range(4)]
+    du = [np.empty_like(x) for _ in range(4)]
+    arr4 = _dp * 4
+    rc = _load().gspn_oracle_backward(_ptr(x), arr4(*[_ptr(a) for a in zs]),
+                                      arr4(*[_ptr(a) for a in ls]), arr4(*[_ptr(a) for a in us]),
+                                      _ptr(gy), B, C, H, W, int(group_len), int(nthreads),
+                                      _ptr(dx), arr4(*[_ptr(a) for a in dz]),
+                                      arr4(*[_ptr(a) for a in dl]), arr4(*[_ptr(a) for a in du]))
+    if rc != 0:
+        raise ValueError(f"oracle rejected arguments (rc={rc})")
+    return dx, dz, dl, du

@@ -35,6 +35,19 @@
 //
 // Layouts (contiguous, row-major): x, lam[d], u[d], y: [B][C][H][W];
 // wlogit[d]: [B][C][3][H][W].  All arrays are double.
+//
+// Backward (section "反向传播" of the same walkthrough: the gradient flows
+// into each line's hidden state from the later lines of the scan, and the
+// input and gate gradients follow from it and the previous hidden state).
+// For L = sum(gy (.) y) the adjoint a_i = dL/dh_i of one direction obeys
+//     a_i = u_i (.) gy_i + w_{i+1}^T a_{i+1}      (no second term when line
+//                                                   i+1 starts a group)
+// and  dx = sum_d lambda_d (.) a_d,  dlambda_d = x (.) a_d,  du_d = gy (.) h_d,
+//      dW_i[k,o] = a_i[k] h_{i-1}[k+o]  (lines that do not start a group),
+// and, through w_o = s_o / sum_p s_p with s = sigmoid(z) over the existing
+// neighbours,  dz_p = w_p (1 - s_p) (dW_p - sum_o dW_o w_o)  (0 for a missing
+// neighbour and on a group's first line).  This is the chain rule on the
+// forward definition above; the pages' own backward stops at the gates.
 
 #include <cmath>
 #include <cstdint>
@@ -112,6 +125,55 @@ void plane_hidden(const Dir& dir, const double* x, const double* z3, const doubl
             h[p] = cur[k];
         }
         prev.swap(cur);
+    }
+}
+
+// Gradients of L = sum(gy (.) y) with respect to the inputs of one plane and
+// one direction: dx is accumulated, dz3, dlam and du are written.  h is
+// scratch of H*W doubles.
+void plane_backward(const Dir& dir, const double* x, const double* z3, const double* lam,
+                    const double* u, const double* gy, int64_t g, double* dx, double* dz3,
+                    double* dlam, double* du, double* h) {
+    const int64_t L = dir.L(), K = dir.K(), HW = dir.H * dir.W;
+    plane_hidden(dir, x, z3, lam, g, h);
+    std::vector<double> a(K), carry(K, 0.0);
+    for (int64_t i = L - 1; i >= 0; --i) {
+        const bool start = group_start(dir, i, g);
+        for (int64_t k = 0; k < K; ++k) {
+            const int64_t p = dir.pixel(i, k);
+            a[k] = u[p] * gy[p] + carry[k];
+            du[p] = gy[p] * h[p];
+            dlam[p] = x[p] * a[k];
+            dx[p] += lam[p] * a[k];
+        }
+        for (int64_t k = 0; k < K; ++k) carry[k] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const int64_t p = dir.pixel(i, k);
+            if (start) {
+                for (int slot = 0; slot < 3; ++slot) dz3[slot * HW + p] = 0.0;
+                continue;
+            }
+            double w[3];
+            pixel_weights(z3, HW, p, k, K, w);
+            double dw[3] = {0.0, 0.0, 0.0};
+            double dw_dot_w = 0.0;
+            for (int slot = 0; slot < 3; ++slot) {
+                const int64_t kn = k + slot - 1;
+                if (kn < 0 || kn >= K) continue;
+                dw[slot] = a[k] * h[dir.pixel(i - 1, kn)];
+                dw_dot_w += dw[slot] * w[slot];
+                carry[kn] += w[slot] * a[k];
+            }
+            for (int slot = 0; slot < 3; ++slot) {
+                const int64_t kn = k + slot - 1;
+                if (kn < 0 || kn >= K) {
+                    dz3[slot * HW + p] = 0.0;
+                    continue;
+                }
+                const double sg = logistic(z3[slot * HW + p]);
+                dz3[slot * HW + p] = w[slot] * (1.0 - sg) * (dw[slot] - dw_dot_w);
+            }
+        }
     }
 }
 
@@ -199,6 +261,33 @@ int gspn_oracle_forward(const double* x, const double* const* wlogit, const doub
                          h.data());
             const double* ud = u[d] + q * HW;
             for (int64_t p = 0; p < HW; ++p) yq[p] += ud[p] * h[p];
+        }
+    });
+    return 0;
+}
+
+// Gradients of L = sum(gy (.) y) for the four-direction operation:
+// dx[B][C][H][W]; dwlogit[d][B][C][3][H][W]; dlam[d], du[d][B][C][H][W].
+// Returns 0, or -1 on a bad argument.
+int gspn_oracle_backward(const double* x, const double* const* wlogit, const double* const* lam,
+                         const double* const* u, const double* gy, int64_t B, int64_t C,
+                         int64_t H, int64_t W, int64_t group_len, int nthreads, double* dx,
+                         double* const* dwlogit, double* const* dlam, double* const* du) {
+    if (!x || !wlogit || !lam || !u || !gy || !dx || !dwlogit || !dlam || !du ||
+        bad_shape(B, C, H, W) || group_len < 0)
+        return -1;
+    for (int d = 0; d < 4; ++d)
+        if (!wlogit[d] || !lam[d] || !u[d] || !dwlogit[d] || !dlam[d] || !du[d]) return -1;
+    const int64_t HW = H * W;
+    parallel_planes(B * C, nthreads, [&](int64_t q) {
+        std::vector<double> h(HW);
+        double* dxq = dx + q * HW;
+        for (int64_t p = 0; p < HW; ++p) dxq[p] = 0.0;
+        for (int d = 0; d < 4; ++d) {
+            const Dir dir{d, H, W};
+            plane_backward(dir, x + q * HW, wlogit[d] + q * 3 * HW, lam[d] + q * HW,
+                           u[d] + q * HW, gy + q * HW, group_len, dxq, dwlogit[d] + q * 3 * HW,
+                           dlam[d] + q * HW, du[d] + q * HW, h.data());
         }
     });
     return 0;

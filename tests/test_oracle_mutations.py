@@ -35,6 +35,14 @@ MUTATIONS = [
      "case 2: return k * W + i;", "case 2: return k * W + (W - 1 - i);"),
     ("u of the wrong direction",
      "const double* ud = u[d] + q * HW;", "const double* ud = u[(d + 1) % 4] + q * HW;"),
+    # backward
+    ("sigmoid derivative factor dropped",
+     "dz3[slot * HW + p] = w[slot] * (1.0 - sg) * (dw[slot] - dw_dot_w);",
+     "dz3[slot * HW + p] = w[slot] * (dw[slot] - dw_dot_w);"),
+    ("adjoint carried to the wrong neighbour",
+     "carry[kn] += w[slot] * a[k];", "carry[k] += w[slot] * a[k];"),
+    ("gate gradient uses the current line",
+     "dw[slot] = a[k] * h[dir.pixel(i - 1, kn)];", "dw[slot] = a[k] * h[dir.pixel(i, kn)];"),
 ]
 
 
@@ -47,8 +55,8 @@ def _run_pins_on_copy(tmp_path, src):
     (tmp_path / "oracle" / "gspn_oracle.cpp").write_text(src)
     env = dict(os.environ, PYTHONPATH=str(tmp_path))
     return subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                           "tests/test_oracle_pins.py"], cwd=tmp_path, env=env,
-                          capture_output=True, text=True, timeout=600)
+                           "tests/test_oracle_pins.py", "tests/test_oracle_backward_pins.py"],
+                          cwd=tmp_path, env=env, capture_output=True, text=True, timeout=600)
 
 
 def test_unmodified_copy_passes(tmp_path):
