@@ -108,6 +108,25 @@ int gspn_forward_host(const void* x, const void* const wlogit[4], const void* co
                       int64_t group_len, int dtype, void* stream, void* y);
 
 /*
+ * Backward pass (walkthrough section "反向传播"): the gradients of
+ * L = sum(gy (.) y) with respect to every input of gspn_forward, where y is
+ * gspn_forward's output for the same arguments.
+ *   dx[B][C][H][W]; dwlogit[d][B][C][3][H][W] (through the sigmoid and the
+ *   border-aware normalisation; 0 for a missing neighbour and on a group's
+ *   first line); dlam[d], du[d][B][C][H][W].
+ * Same layouts, dtype, alignment and stream rules as gspn_forward; outputs
+ * are device memory owned by the caller, overwritten completely, and must
+ * not overlap any input or each other (GSPN_ERR_ALIAS).  Arithmetic is fp32;
+ * each output is rounded once to the storage dtype.  The library keeps a
+ * per-device fp32 workspace of 5 * B*C*H*W floats for it (freed by
+ * gspn_release).
+ */
+int gspn_backward(const void* x, const void* const wlogit[4], const void* const lam[4],
+                  const void* const u[4], const void* gy, int64_t B, int64_t C, int64_t H,
+                  int64_t W, int64_t group_len, int dtype, void* stream, void* dx,
+                  void* const dwlogit[4], void* const dlam[4], void* const du[4]);
+
+/*
  * gspn_forward without any device allocation.  The operation has no
  * counterpart in the GSPN papers or pages: it is a deployment variant of the
  * same computation for callers that cannot call cudaMalloc when they run it

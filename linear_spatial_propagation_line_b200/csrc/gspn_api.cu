@@ -24,6 +24,8 @@ struct DeviceBuffers {
     bool pending_error = false;  // a device error seen while replacing the workspace
     void* staging = nullptr;
     size_t staging_bytes = 0;
+    void* bws = nullptr;  // backward: hidden states and the dx accumulator
+    size_t bws_bytes = 0;
 };
 
 std::mutex g_mutex;
@@ -304,6 +306,76 @@ int gspn_forward_noalloc(const void* x, const void* const wlogit[4], const void*
     return GSPN_OK;
 }
 
+int gspn_backward(const void* x, const void* const wlogit[4], const void* const lam[4],
+                  const void* const u[4], const void* gy, int64_t B, int64_t C, int64_t H,
+                  int64_t W, int64_t group_len, int dtype, void* stream, void* dx,
+                  void* const dwlogit[4], void* const dlam[4], void* const du[4]) {
+    if (!gy || !dx || !dwlogit || !dlam || !du) return GSPN_ERR_NULL;
+    for (int d = 0; d < 4; ++d)
+        if (!dwlogit[d] || !dlam[d] || !du[d]) return GSPN_ERR_NULL;
+    gspn::BackwardProblem bp;
+    // validate the forward inputs; dx stands in for y in the alias checks
+    int s = validate(x, wlogit, lam, u, B, C, H, W, group_len, dtype, 0, 4, true, dx, &bp.fwd);
+    if (s != GSPN_OK) return s;
+    if (!aligned16(gy)) return GSPN_ERR_ALIGN;
+    for (int d = 0; d < 4; ++d)
+        if (!aligned16(dwlogit[d]) || !aligned16(dlam[d]) || !aligned16(du[d]))
+            return GSPN_ERR_ALIGN;
+    // no output may overlap an input or another output
+    const size_t es = dtype == GSPN_F32 ? 4 : 2;
+    const size_t n = (size_t)(B * C * H * W) * es;
+    const void* in_p[14];
+    size_t in_n[14];
+    int ni = 0;
+    in_p[ni] = x; in_n[ni++] = n;
+    in_p[ni] = gy; in_n[ni++] = n;
+    for (int d = 0; d < 4; ++d) {
+        in_p[ni] = wlogit[d]; in_n[ni++] = 3 * n;
+        in_p[ni] = lam[d]; in_n[ni++] = n;
+        in_p[ni] = u[d]; in_n[ni++] = n;
+    }
+    const void* out_p[13];
+    size_t out_n[13];
+    int no = 0;
+    out_p[no] = dx; out_n[no++] = n;
+    for (int d = 0; d < 4; ++d) {
+        out_p[no] = dwlogit[d]; out_n[no++] = 3 * n;
+        out_p[no] = dlam[d]; out_n[no++] = n;
+        out_p[no] = du[d]; out_n[no++] = n;
+    }
+    for (int o = 0; o < no; ++o) {
+        for (int i = 0; i < ni; ++i)
+            if (overlaps(out_p[o], out_n[o], in_p[i], in_n[i])) return GSPN_ERR_ALIAS;
+        for (int o2 = o + 1; o2 < no; ++o2)
+            if (overlaps(out_p[o], out_n[o], out_p[o2], out_n[o2])) return GSPN_ERR_ALIAS;
+    }
+    bp.gy = gy;
+    bp.dx = dx;
+    for (int d = 0; d < 4; ++d) {
+        bp.dz[d] = dwlogit[d];
+        bp.dlam[d] = dlam[d];
+        bp.du[d] = du[d];
+    }
+    bp.fwd.stream = static_cast<cudaStream_t>(stream);
+    bp.fwd.ev_begin = t_ev_begin;
+    bp.fwd.ev_end = t_ev_end;
+    int dev;
+    if ((s = current_device(&dev)) != GSPN_OK) return s;
+    int launches = 0;
+    cudaError_t e;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        DeviceBuffers& db = g_dev[dev];
+        s = ensure_buffer(&db.bws, &db.bws_bytes, gspn::backward_workspace_bytes(bp.fwd));
+        if (s != GSPN_OK) return s;
+        e = gspn::launch_backward(bp, static_cast<float*>(db.bws), &launches);
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    t_last_launches = launches;
+    t_last_kernel = bp.fwd.kernel_name;
+    return GSPN_OK;
+}
+
 int gspn_last_launch_count(void) { return t_last_launches; }
 
 int gspn_check_device_status(void* stream) {
@@ -363,6 +435,10 @@ int gspn_release(void) {
     }
     if (db.staging) {
         cudaError_t e2 = cudaFree(db.staging);
+        if (e == cudaSuccess) e = e2;
+    }
+    if (db.bws) {
+        cudaError_t e2 = cudaFree(db.bws);
         if (e == cudaSuccess) e = e2;
     }
     db = DeviceBuffers();

@@ -42,6 +42,20 @@ cudaError_t launch_small_plane(Problem& pb, int* launches);
 // writes y.
 cudaError_t launch_chain(Problem& pb, float* ws, int* launches);
 
+// Backward pass: gradients of L = sum(gy * y) for every input of a forward
+// call.  Workspace: backward_workspace_bytes(fwd) bytes of fp32 (every
+// direction's hidden state and the dx accumulator).
+struct BackwardProblem {
+    Problem fwd;          // the forward call's inputs (all four directions)
+    const void* gy;       // dL/dy [B][C][H][W]
+    void* dx;             // [B][C][H][W]
+    void* dz[4];          // [B][C][3][H][W]
+    void* dlam[4];        // [B][C][H][W]
+    void* du[4];          // [B][C][H][W]
+};
+size_t backward_workspace_bytes(const Problem& pb);
+cudaError_t launch_backward(BackwardProblem& bp, float* ws, int* launches);
+
 // Fixed-scratch variant of the line-chain path (gspn_forward_noalloc): the
 // fp32 accumulator is a static device array of kNoAllocMaxPixch floats.
 // noalloc_scratch returns its address on `device` (which must be current),

@@ -56,6 +56,9 @@ def load_library():
         lib.gspn_forward_host.argtypes = [vp, arr4, arr4, arr4, i64, i64, i64, i64, i64, ci, vp,
                                           vp]
         lib.gspn_forward_host.restype = ci
+        lib.gspn_backward.argtypes = [vp, arr4, arr4, arr4, vp, i64, i64, i64, i64, i64, ci, vp,
+                                      vp, arr4, arr4, arr4]
+        lib.gspn_backward.restype = ci
         lib.gspn_forward_noalloc.argtypes = [vp, arr4, arr4, arr4, i64, i64, i64, i64, i64, ci,
                                              vp, vp]
         lib.gspn_forward_noalloc.restype = ci
@@ -201,6 +204,56 @@ def forward_noalloc(x, wlogit, lam, u, group_len: int = 0, out=None, stream=None
                                         arr4(*[t.data_ptr() for t in u]), B, C, H, W,
                                         int(group_len), _DTYPES[x.dtype], st, y.data_ptr()))
     return y
+
+
+def backward(x, wlogit, lam, u, gy, group_len: int = 0, stream=None):
+    """Gradients of sum(gy * forward(x, wlogit, lam, u)) with respect to every
+    input, on CUDA tensors: returns (dx, [dwlogit_d], [dlam_d], [du_d])."""
+    lib = load_library()
+    B, C, H, W = _validate(x, wlogit, lam, u, range(4), "cuda")
+    _validate(gy, wlogit, lam, u, [], "cuda")
+    if gy.dtype != x.dtype or tuple(gy.shape) != tuple(x.shape) or not gy.is_contiguous():
+        raise ValueError("gy must be a contiguous tensor like x")
+    dx = torch.empty_like(x)
+    dz = [torch.empty_like(t) for t in wlogit]
+    dl = [torch.empty_like(t) for t in lam]
+    du = [torch.empty_like(t) for t in u]
+    arr4 = ctypes.c_void_p * 4
+    with torch.cuda.device(x.device):
+        st = _stream_handle(x.device, stream)
+        _check(lib.gspn_backward(x.data_ptr(), arr4(*[t.data_ptr() for t in wlogit]),
+                                 arr4(*[t.data_ptr() for t in lam]),
+                                 arr4(*[t.data_ptr() for t in u]), gy.data_ptr(), B, C, H, W,
+                                 int(group_len), _DTYPES[x.dtype], st, dx.data_ptr(),
+                                 arr4(*[t.data_ptr() for t in dz]),
+                                 arr4(*[t.data_ptr() for t in dl]),
+                                 arr4(*[t.data_ptr() for t in du])))
+    return dx, dz, dl, du
+
+
+class GSPNFunction(torch.autograd.Function):
+    """Autograd wrapper: forward() runs gspn_forward, backward() gspn_backward.
+    Inputs: x, then the four logits, the four lambdas, the four u tensors."""
+
+    @staticmethod
+    def forward(ctx, group_len, x, *params):
+        wlogit, lam, u = list(params[0:4]), list(params[4:8]), list(params[8:12])
+        ctx.group_len = int(group_len)
+        ctx.save_for_backward(x, *params)
+        return forward(x.contiguous(), [t.contiguous() for t in wlogit],
+                       [t.contiguous() for t in lam], [t.contiguous() for t in u], group_len)
+
+    @staticmethod
+    def backward(ctx, gy):
+        x, *params = ctx.saved_tensors
+        wlogit, lam, u = list(params[0:4]), list(params[4:8]), list(params[8:12])
+        dx, dz, dl, du = backward(x, wlogit, lam, u, gy.contiguous(), ctx.group_len)
+        return (None, dx, *dz, *dl, *du)
+
+
+def gspn_autograd(x, wlogit, lam, u, group_len: int = 0):
+    """y = sum_d u_d * h_d with gradients for every input (torch autograd)."""
+    return GSPNFunction.apply(int(group_len), x, *wlogit, *lam, *u)
 
 
 def forward_dir(x, wlogit_d, lam_d, u_d, d: int, group_len: int = 0, out=None, stream=None):
