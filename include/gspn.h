@@ -86,6 +86,18 @@ int gspn_forward(const void* x, const void* const wlogit[4], const void* const l
                  int64_t group_len, int dtype, void* stream, void* y);
 
 /*
+ * gspn_forward with channel-shared neighbour logits: wlogit[d] is
+ * [B][1][3][H][W] and every channel c of batch entry b uses the logits of b.
+ * lam[d], u[d], x and y keep their [B][C][H][W] layout.  This is the plain
+ * reading of the walkthrough's section "局限性" (the feature dimension of the
+ * propagation weights set to 1 to fit memory); it moves 10 + 12/C elements per
+ * pixel-channel instead of 22.  Same rules and errors as gspn_forward.
+ */
+int gspn_forward_shared(const void* x, const void* const wlogit[4], const void* const lam[4],
+                        const void* const u[4], int64_t B, int64_t C, int64_t H, int64_t W,
+                        int64_t group_len, int dtype, void* stream, void* y);
+
+/*
  * One direction only: y = u (.) h_d(x; wlogit, lam, group_len), with the
  * same layouts, rules and errors as gspn_forward (d in 0..3, else
  * GSPN_ERR_DIR).  Used to test each scan direction on its own.

@@ -98,7 +98,7 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 int validate(const void* x, const void* const* wlogit, const void* const* lam,
              const void* const* u, int64_t B, int64_t C, int64_t H, int64_t W,
              int64_t group_len, int dtype, int d0, int d1, bool need_align, void* y,
-             gspn::Problem* pb) {
+             gspn::Problem* pb, bool shared_logits = false) {
     if (!x || !wlogit || !lam || !u || !y) return GSPN_ERR_NULL;
     for (int d = d0; d < d1; ++d)
         if (!wlogit[d] || !lam[d] || !u[d]) return GSPN_ERR_NULL;
@@ -115,8 +115,9 @@ int validate(const void* x, const void* const* wlogit, const void* const* lam,
     const size_t es = dtype == GSPN_F32 ? 4 : 2;
     const size_t n = (size_t)(B * C * H * W) * es;
     if (overlaps(y, n, x, n)) return GSPN_ERR_ALIAS;
+    const size_t nz = shared_logits ? (size_t)(B * H * W) * es : n;  // one logit plane set per b
     for (int d = d0; d < d1; ++d)
-        if (overlaps(y, n, wlogit[d], 3 * n) || overlaps(y, n, lam[d], n) ||
+        if (overlaps(y, n, wlogit[d], 3 * nz) || overlaps(y, n, lam[d], n) ||
             overlaps(y, n, u[d], n))
             return GSPN_ERR_ALIAS;
     pb->x = x;
@@ -131,6 +132,7 @@ int validate(const void* x, const void* const* wlogit, const void* const* lam,
     pb->H = H;
     pb->W = W;
     pb->g = group_len > 0x7fffffffLL ? 0x7fffffffLL : group_len;
+    pb->z_div = shared_logits ? C : 1;
     pb->dtype = dtype;
     pb->d0 = d0;
     pb->d1 = d1;
@@ -214,6 +216,16 @@ int gspn_forward(const void* x, const void* const wlogit[4], const void* const l
                  int64_t group_len, int dtype, void* stream, void* y) {
     gspn::Problem pb;
     int s = validate(x, wlogit, lam, u, B, C, H, W, group_len, dtype, 0, 4, true, y, &pb);
+    if (s != GSPN_OK) return s;
+    pb.stream = static_cast<cudaStream_t>(stream);
+    return run(pb);
+}
+
+int gspn_forward_shared(const void* x, const void* const wlogit[4], const void* const lam[4],
+                        const void* const u[4], int64_t B, int64_t C, int64_t H, int64_t W,
+                        int64_t group_len, int dtype, void* stream, void* y) {
+    gspn::Problem pb;
+    int s = validate(x, wlogit, lam, u, B, C, H, W, group_len, dtype, 0, 4, true, y, &pb, true);
     if (s != GSPN_OK) return s;
     pb.stream = static_cast<cudaStream_t>(stream);
     return run(pb);

@@ -18,7 +18,7 @@ constexpr int kThreads = 512;
 template <class T, bool kRefine>
 __global__ void __launch_bounds__(kThreads)
     chain_kernel(const T* __restrict__ x, Ptr4 zp, Ptr4 lp, Ptr4 up, int H, int W, int g,
-                 int d0, float* __restrict__ ws) {
+                 int d0, int z_div, float* __restrict__ ws) {
     extern __shared__ __align__(16) float hb[];
     const int d = d0 + (int)blockIdx.y;
     const int64_t plane = blockIdx.x;
@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(kThreads)
     const int L = vert ? H : W;
     const int K = vert ? W : H;
     const T* xq = x + plane * HW;
-    const T* zq = static_cast<const T*>(zp.p[d]) + plane * 3 * HW;
+    const T* zq = static_cast<const T*>(zp.p[d]) + (plane / z_div) * 3 * HW;
     const T* lq = static_cast<const T*>(lp.p[d]) + plane * HW;
     const T* uq = static_cast<const T*>(up.p[d]) + plane * HW;
     float* wq = ws + plane * HW;
@@ -82,7 +82,7 @@ cudaError_t launch_typed(Problem& pb, float* ws, int* launches) {
     dim3 grid((unsigned)pb.planes(), (unsigned)(pb.d1 - pb.d0));
     if (pb.ev_begin) cudaEventRecord(pb.ev_begin, pb.stream);
     kernel<<<grid, kThreads, smem, pb.stream>>>(static_cast<const T*>(pb.x), pb.z, pb.lam, pb.u,
-                                                H, W, (int)pb.g, pb.d0, ws);
+                                                H, W, (int)pb.g, pb.d0, (int)pb.z_div, ws);
     if (pb.ev_end) cudaEventRecord(pb.ev_end, pb.stream);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     convert_kernel<T><<<148 * 8, 256, 0, pb.stream>>>(ws, pb.pixch(), static_cast<T*>(pb.y));

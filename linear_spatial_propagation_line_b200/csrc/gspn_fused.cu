@@ -99,6 +99,7 @@ struct __align__(64) FusedParams {
     int nb_h, bh_h;        // horizontal: row boxes, box height (multiple of 8)
     int tile_bytes;        // one tensor's tile in one stage
     int stages;            // depth of the shared-memory ring (2 or 3)
+    int z_div;             // logits of plane q are logit plane q / z_div
     int n_slots;
     int n_items;
     int force_stale;       // test hook: expect a slot epoch that never comes
@@ -485,8 +486,8 @@ __device__ __forceinline__ const CUtensorMap* tensor_map(const FusedParams& p,
                                                          int tensor) {
     return tensor == 0 ? xmap : tensor <= 3 ? &p.tm_z[d] : tensor == 4 ? &p.tm_l[d] : &p.tm_u[d];
 }
-__device__ __forceinline__ int tensor_z(int q, int tensor) {
-    return tensor == 0 ? q : tensor <= 3 ? 3 * q + tensor - 1 : q;
+__device__ __forceinline__ int tensor_z(const FusedParams& p, int q, int tensor) {
+    return tensor == 0 ? q : tensor <= 3 ? 3 * (q / p.z_div) + tensor - 1 : q;
 }
 
 // ------------------------------------------------------------------- one chain
@@ -797,9 +798,9 @@ __device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& 
                              const CUtensorMap* map = tensor_map(p, &p.tm_xv, d, tensor);
                              if (tensor == 0)
                                  ptx::tma_load_3d_normal(dst, map, kb + 64 * b, row0,
-                                                         tensor_z(q, tensor), bar);
+                                                         tensor_z(p, q, tensor), bar);
                              else
-                                 ptx::tma_load_3d(dst, map, kb + 64 * b, row0, tensor_z(q, tensor),
+                                 ptx::tma_load_3d(dst, map, kb + 64 * b, row0, tensor_z(p, q, tensor),
                                                   bar, pol_in);
                          });
         } else {
@@ -809,7 +810,7 @@ __device__ __forceinline__ void run_chain(const FusedParams& p, const SmemView& 
                              const int col0 = FWD ? st * kSeg : W - kSeg - st * kSeg;
                              const uint32_t dst = ptx::smem_addr(sm.tile(sl, tensor)) + b * bh * 32;
                              ptx::tma_load_3d_normal(dst, tensor_map(p, &p.tm_xh, d, tensor), col0,
-                                                     kb + b * bh, tensor_z(q, tensor), bar);
+                                                     kb + b * bh, tensor_z(p, q, tensor), bar);
                          });
         }
     } else if (t < nthr) {
@@ -1110,7 +1111,8 @@ cudaError_t launch_typed(Problem& pb, const FusedPlan& fp, void* ws) {
         const bool vert = d < 2;
         const int bx = vert ? 64 : J;
         const int by = vert ? J : fp.bh_h;
-        if (!encode_map(&prm.tm_z[d], pb.z.p[d], pb.dtype, W, H, 3 * planes, bx, by, !vert) ||
+        if (!encode_map(&prm.tm_z[d], pb.z.p[d], pb.dtype, W, H, 3 * (planes / pb.z_div), bx, by,
+                        !vert) ||
             !encode_map(&prm.tm_l[d], pb.lam.p[d], pb.dtype, W, H, planes, bx, by, !vert) ||
             !encode_map(&prm.tm_u[d], pb.u.p[d], pb.dtype, W, H, planes, bx, by, !vert))
             return cudaErrorInvalidValue;
@@ -1139,6 +1141,7 @@ cudaError_t launch_typed(Problem& pb, const FusedPlan& fp, void* ws) {
     prm.stages = fp.stages;
     prm.n_slots = fp.n_slots;
     prm.n_items = (int)(planes * nd);
+    prm.z_div = (int)pb.z_div;
     prm.force_stale = fp.force_stale;
 
     // Reset the per-call part of the control block (not the sticky error).

@@ -20,6 +20,7 @@ struct Problem {
     Ptr4 lam;  // [B][C][H][W]
     Ptr4 u;    // [B][C][H][W]
     int64_t B, C, H, W, g;
+    int64_t z_div = 1;  // logits of plane q are logit plane q / z_div (C: shared by channels)
     int dtype;  // GSPN_F32 / GSPN_BF16
     int d0, d1;
     cudaStream_t stream;

@@ -45,7 +45,7 @@ SmallLayout small_layout(int H, int W) {
 template <class T, bool kRefine, int V>
 __global__ void __launch_bounds__(kThreads)
     small_plane_kernel(const T* __restrict__ x, Ptr4 zp, Ptr4 lp, Ptr4 up, int H, int W, int g,
-                       int d0, int d1, int pitch_y, int kp_v, int kp_h, int scr,
+                       int d0, int d1, int pitch_y, int kp_v, int kp_h, int scr, int z_div,
                        T* __restrict__ y) {
     extern __shared__ __align__(16) float smem[];
     float* yacc = smem;
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kThreads)
     for (int p = threadIdx.x; p < H * pitch_y; p += kThreads) yacc[p] = 0.0f;
 
     for (int d = d0; d < d1; ++d) {
-        const T* zq = static_cast<const T*>(zp.p[d]) + plane * 3 * HW;
+        const T* zq = static_cast<const T*>(zp.p[d]) + (plane / z_div) * 3 * HW;
         const T* lq = static_cast<const T*>(lp.p[d]) + plane * HW;
         const T* uq = static_cast<const T*>(up.p[d]) + plane * HW;
         const bool vert = d < 2;
@@ -160,7 +160,7 @@ cudaError_t launch_typed(const Problem& pb) {
         if (pb.ev_begin) cudaEventRecord(pb.ev_begin, pb.stream);
         kernel<<<(unsigned)pb.planes(), kThreads, s.bytes, pb.stream>>>(
             static_cast<const T*>(pb.x), pb.z, pb.lam, pb.u, H, W, (int)pb.g, pb.d0, pb.d1,
-            s.pitch_y, s.kp_v, s.kp_h, s.scr, static_cast<T*>(pb.y));
+            s.pitch_y, s.kp_v, s.kp_h, s.scr, (int)pb.z_div, static_cast<T*>(pb.y));
         if (pb.ev_end) cudaEventRecord(pb.ev_end, pb.stream);
         return cudaGetLastError();
     };

@@ -56,6 +56,9 @@ def load_library():
         lib.gspn_forward_host.argtypes = [vp, arr4, arr4, arr4, i64, i64, i64, i64, i64, ci, vp,
                                           vp]
         lib.gspn_forward_host.restype = ci
+        lib.gspn_forward_shared.argtypes = [vp, arr4, arr4, arr4, i64, i64, i64, i64, i64, ci,
+                                            vp, vp]
+        lib.gspn_forward_shared.restype = ci
         lib.gspn_backward.argtypes = [vp, arr4, arr4, arr4, vp, i64, i64, i64, i64, i64, ci, vp,
                                       vp, arr4, arr4, arr4]
         lib.gspn_backward.restype = ci
@@ -203,6 +206,32 @@ def forward_noalloc(x, wlogit, lam, u, group_len: int = 0, out=None, stream=None
                                         arr4(*[t.data_ptr() for t in lam]),
                                         arr4(*[t.data_ptr() for t in u]), B, C, H, W,
                                         int(group_len), _DTYPES[x.dtype], st, y.data_ptr()))
+    return y
+
+
+def forward_shared(x, wlogit, lam, u, group_len: int = 0, out=None, stream=None):
+    """forward() with channel-shared logits: wlogit[d] is [B,1,3,H,W]."""
+    lib = load_library()
+    B, C, H, W = _shape_of(x)
+    for d in range(4):
+        if tuple(wlogit[d].shape) != (B, 1, 3, H, W):
+            raise ValueError(f"wlogit[{d}] must be [B,1,3,H,W], got {tuple(wlogit[d].shape)}")
+    # the per-channel checks of _validate on a broadcast view of the logits
+    _validate(x, [t.expand(B, C, 3, H, W) for t in wlogit], lam, u, [], "cuda")
+    for t in list(wlogit) + list(lam) + list(u):
+        if t.dtype != x.dtype or not t.is_contiguous() or not t.is_cuda or t.device != x.device:
+            raise ValueError("every tensor must be contiguous, on x's device, with x's dtype")
+    for d in range(4):
+        if tuple(lam[d].shape) != (B, C, H, W) or tuple(u[d].shape) != (B, C, H, W):
+            raise ValueError("lam[d], u[d] must be [B,C,H,W]")
+    y = torch.empty_like(x) if out is None else out
+    arr4 = ctypes.c_void_p * 4
+    with torch.cuda.device(x.device):
+        st = _stream_handle(x.device, stream)
+        _check(lib.gspn_forward_shared(x.data_ptr(), arr4(*[t.data_ptr() for t in wlogit]),
+                                       arr4(*[t.data_ptr() for t in lam]),
+                                       arr4(*[t.data_ptr() for t in u]), B, C, H, W,
+                                       int(group_len), _DTYPES[x.dtype], st, y.data_ptr()))
     return y
 
 
