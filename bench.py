@@ -47,6 +47,7 @@ KERNELS = {
     "small_plane_kernel": (["gspn_small.cu", "gspn_common.cuh"], 22),
     "chain_kernel": (["gspn_chain.cu", "gspn_common.cuh"], 21),
     "fused_kernel": (["gspn_fused.cu", "gspn_ptx.cuh", "gspn_common.cuh"], 22),
+    "sweep_kernel": (["gspn_sweep.cu", "gspn_ptx.cuh", "gspn_common.cuh"], 22),
 }
 CSRC = ROOT / "linear_spatial_propagation_line_b200" / "csrc"
 
@@ -63,6 +64,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["auto", "fused", "sweep"], default="auto",
+                    help="large-plane kernel (auto: the fused kernel)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -284,6 +287,8 @@ def run_ours(args, wl):
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     gspn.load_library()
+    gspn.debug_select_path({"auto": gspn.PATH_AUTO, "fused": gspn.PATH_FUSED,
+                            "sweep": gspn.PATH_SWEEP}[args.path])
 
     inp = make_inputs(wl, seed=rank, device=str(device), gen_device=str(device))
     y = torch.empty_like(inp["x"])

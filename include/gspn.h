@@ -200,6 +200,20 @@ int gspn_check_device_status(void* stream);
  */
 int gspn_debug_force_timeout(int64_t timeout_ns);
 
+/*
+ * Test hook: which kernel takes large planes on this thread from now on.
+ * GSPN_PATH_AUTO (the default) and GSPN_PATH_FUSED use the fused kernel and
+ * fall back to the line-chain kernel when a plane does not fit its
+ * constraints; GSPN_PATH_SWEEP uses the line-sweep kernel (scan line in
+ * registers, warp-shuffle neighbours) instead of the fused kernel.  Results
+ * agree within the tolerances of the storage dtype.  Returns GSPN_OK, or
+ * GSPN_ERR_DIR for an unknown path.
+ */
+#define GSPN_PATH_AUTO 0
+#define GSPN_PATH_FUSED 1
+#define GSPN_PATH_SWEEP 2
+int gspn_debug_select_path(int path);
+
 /* Frees the current device's workspace and staging area.  Not thread safe
  * against concurrent gspn_* calls on the same device. */
 int gspn_release(void);

@@ -38,6 +38,7 @@ thread_local cudaEvent_t t_ev_end = nullptr;
 thread_local const char* t_last_kernel = "";
 thread_local bool t_force_timeout = false;
 thread_local unsigned long long t_force_timeout_ns = 0;
+thread_local int t_large_path = GSPN_PATH_AUTO;
 
 int cuda_fail(cudaError_t e) {
     snprintf(t_cuda_error, sizeof(t_cuda_error), "%s: %s", cudaGetErrorName(e),
@@ -173,9 +174,26 @@ int run(gspn::Problem& pb) {
     pb.ev_end = t_ev_end;
     cudaError_t e;
     gspn::FusedPlan fp;
+    gspn::SweepPlan sp;
     if (gspn::small_plane_fits(pb, nullptr)) {
         e = gspn::launch_small_plane(pb, &launches);
-    } else if (gspn::fused_plan(pb, &fp)) {
+    } else if (t_large_path == GSPN_PATH_SWEEP && gspn::sweep_plan(pb, &sp)) {
+        int dev;
+        int s = current_device(&dev);
+        if (s != GSPN_OK) return s;
+        std::lock_guard<std::mutex> lock(g_mutex);
+        DeviceBuffers& db = g_dev[dev];
+        s = ensure_fused(db, sp.ws_bytes, pb.stream);
+        if (s != GSPN_OK) return s;
+        sp.zero_slots = db.fused_dirty;
+        db.fused_dirty = false;
+        if (t_force_timeout) {
+            sp.force_stale = 1;
+            sp.timeout_ns = t_force_timeout_ns;
+            t_force_timeout = false;
+        }
+        e = gspn::launch_sweep(pb, sp, db.fused, &launches);
+    } else if (t_large_path != GSPN_PATH_SWEEP && gspn::fused_plan(pb, &fp)) {
         int dev;
         int s = current_device(&dev);
         if (s != GSPN_OK) return s;
@@ -422,6 +440,13 @@ int gspn_debug_force_timeout(int64_t timeout_ns) {
     if (timeout_ns <= 0) return GSPN_ERR_SHAPE;
     t_force_timeout = true;
     t_force_timeout_ns = (unsigned long long)timeout_ns;
+    return GSPN_OK;
+}
+
+int gspn_debug_select_path(int path) {
+    if (path != GSPN_PATH_AUTO && path != GSPN_PATH_FUSED && path != GSPN_PATH_SWEEP)
+        return GSPN_ERR_DIR;
+    t_large_path = path;
     return GSPN_OK;
 }
 

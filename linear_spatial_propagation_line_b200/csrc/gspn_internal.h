@@ -80,6 +80,27 @@ struct FusedPlan {
 };
 bool fused_plan(const Problem& pb, FusedPlan* fp);
 cudaError_t launch_fused(Problem& pb, const FusedPlan& fp, void* ws, int* launches);
+// Line-sweep persistent path (large planes whose rows are 16-byte multiples):
+// the scan line lives in registers, four positions per lane; one launch
+// computes all directions into the same workspace layout as the fused path.
+struct SweepPlan {
+    int S;                    // CTAs per team (cluster)
+    int So[2], Kc[2];         // CTAs per chain and owned positions per CTA (vertical, horizontal)
+    int nw, threads;          // consumer warps, threads per CTA
+    int nb[2], bw[2];         // boxes per tensor and stage, box width in line positions
+    int tile_bytes, stages;
+    size_t smem;
+    int ipp;                  // work items per plane
+    int item_dir[4][2];       // directions of each item (-1: that half of the team idles)
+    int n_teams, n_slots;
+    size_t slot_bytes, ctrl_bytes, ws_bytes;
+    unsigned long long timeout_ns;
+    bool zero_slots;
+    int force_stale;
+};
+bool sweep_plan(const Problem& pb, SweepPlan* sp);
+cudaError_t launch_sweep(Problem& pb, const SweepPlan& sp, void* ws, int* launches);
+
 // Offset of the sticky device error word inside the fused workspace.
 constexpr size_t kFusedStickyErrorOffset = 0;
 

@@ -252,6 +252,29 @@ __device__ __forceinline__ void sts_v2_f32(uint32_t a, float x, float y) {
 __device__ __forceinline__ void sts_f32(uint32_t a, float v) {
     asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
+// 16-byte shared store of four floats.
+__device__ __forceinline__ void sts_v4_f32(uint32_t a, float x, float y, float z, float w) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(x), "f"(y), "f"(z),
+                 "f"(w)
+                 : "memory");
+}
+// Predicated 8-byte shared store (skipped, no branch, when `on` is 0).
+__device__ __forceinline__ void sts_v2_f32_if(bool on, uint32_t a, float x, float y) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %0, 0;\n\t"
+        "@p st.shared.v2.f32 [%1], {%2, %3};\n\t}" ::"r"((uint32_t)on),
+        "r"(a), "f"(x), "f"(y)
+        : "memory");
+}
+// Predicated 16-byte shared store (skipped, no branch, when `on` is 0).
+__device__ __forceinline__ void sts_v4_f32_if(bool on, uint32_t a, float x, float y, float z,
+                                              float w) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %0, 0;\n\t"
+        "@p st.shared.v4.f32 [%1], {%2, %3, %4, %5};\n\t}" ::"r"((uint32_t)on),
+        "r"(a), "f"(x), "f"(y), "f"(z), "f"(w)
+        : "memory");
+}
 // Named barrier over the first `count` threads of the CTA (count % 32 == 0).
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -80,6 +80,8 @@ def load_library():
         lib.gspn_check_device_status.restype = ci
         lib.gspn_debug_force_timeout.argtypes = [i64]
         lib.gspn_debug_force_timeout.restype = ci
+        lib.gspn_debug_select_path.argtypes = [ci]
+        lib.gspn_debug_select_path.restype = ci
         _lib = lib
         return lib
 
@@ -130,6 +132,17 @@ def check_device_status(stream=None, device=None) -> int:
 def debug_force_timeout(timeout_ns: int):
     """Make the next large-plane launch on this thread expire a bounded wait."""
     _check(load_library().gspn_debug_force_timeout(int(timeout_ns)))
+
+
+PATH_AUTO, PATH_FUSED, PATH_SWEEP = 0, 1, 2
+
+
+def debug_select_path(path: int):
+    """Choose the large-plane kernel for later calls on this thread:
+    PATH_AUTO or PATH_FUSED (the fused kernel) or PATH_SWEEP (the line-sweep
+    kernel); planes outside a kernel's constraints fall back to the line-chain
+    kernel."""
+    _check(load_library().gspn_debug_select_path(int(path)))
 
 
 def release():

@@ -82,32 +82,48 @@ TEAM_SHAPES = [(700, 96, 0), (96, 704, 0), (1500, 200, 0), (200, 1504, 0), (2100
                (3000, 256, 0), (1201, 160, 100), (160, 1208, 33), (1100, 1000, 0)]
 
 
+@pytest.fixture
+def fused_path():
+    gspn.debug_select_path(gspn.PATH_FUSED)
+    yield
+    gspn.debug_select_path(gspn.PATH_AUTO)
+
+
 @pytest.mark.parametrize("H,W,g", TEAM_SHAPES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_large_planes_multi_cta_teams(H, W, g, dtype, cuda_device):
+def test_large_planes_multi_cta_teams(H, W, g, dtype, cuda_device, fused_path):
     wl = Workload("team", 1, 2, H, W, g, dtype)
     check(wl, cuda_device, seed=H + 7 * W + g)
+    # the fused kernel takes planes whose rows are whole 32-byte segments
+    es = 4 if dtype == "f32" else 2
+    assert gspn.last_kernel_name() == ("fused_kernel" if (W * es) % 32 == 0 else "chain_kernel")
 
 
-def test_forced_timeout_is_reported_and_recovers(cuda_device):
+@pytest.mark.parametrize("path,kernel", [(1, "fused_kernel"), (2, "sweep_kernel")])
+def test_forced_timeout_is_reported_and_recovers(path, kernel, cuda_device):
     """A slot hand-over that never comes makes the kernel give up after its
     bounded wait; the host sees GSPN_ERR_TIMEOUT and the next call is exact."""
     wl = Workload("timeout", 1, 3, 256, 512, 0, "f32")
     inp = inputs.make_inputs(wl, 6)
     dev = to_dev(inp, cuda_device)
-    assert gspn.check_device_status() == 0
-    gspn.debug_force_timeout(50_000_000)  # 50 ms
-    gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0)
-    assert gspn.last_kernel_name() == "fused_kernel"
-    assert gspn.check_device_status() == -7
-    assert gspn.check_device_status() == 0
-    y = gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0)
-    ref = oracle.forward(inp["x"], inp["wlogit"], inp["lam"], inp["u"], 0)
-    assert rel_err(y, ref) <= TOL["f32"]
-    assert gspn.check_device_status() == 0
+    gspn.debug_select_path(path)
+    try:
+        assert gspn.check_device_status() == 0
+        gspn.debug_force_timeout(50_000_000)  # 50 ms
+        gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0)
+        assert gspn.last_kernel_name() == kernel
+        assert gspn.check_device_status() == -7
+        assert gspn.check_device_status() == 0
+        y = gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0)
+        assert gspn.last_kernel_name() == kernel
+        ref = oracle.forward(inp["x"], inp["wlogit"], inp["lam"], inp["u"], 0)
+        assert rel_err(y, ref) <= TOL["f32"]
+        assert gspn.check_device_status() == 0
+    finally:
+        gspn.debug_select_path(gspn.PATH_AUTO)
 
 
-def test_fused_path_is_used_for_the_headline_shape(cuda_device):
+def test_large_plane_kernel_for_the_headline_shape(cuda_device):
     wl = WORKLOADS[inputs.HEADLINE].with_(C=2)
     dev = to_dev(inputs.make_inputs(wl, 0), cuda_device)
     gspn.forward(dev["x"], dev["wlogit"], dev["lam"], dev["u"], 0)

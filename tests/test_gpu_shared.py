@@ -1,6 +1,6 @@
 """gspn_forward_shared (channel-shared neighbour logits, [B,1,3,H,W]) against
 the fp64 oracle run on the logits broadcast to every channel, on each of the
-three kernels (whole-plane, line-chain, fused)."""
+four kernels (whole-plane, line-chain, fused, line-sweep)."""
 import numpy as np
 import pytest
 import torch
@@ -20,11 +20,22 @@ CASES = [
     (Workload("sh_chain_f32", 1, 3, 70, 131, 0, "f32"), "chain_kernel"),
     (Workload("sh_fused_bf16", 2, 4, 256, 512, 0, "bf16"), "fused_kernel"),
     (Workload("sh_fused_local_f32", 1, 3, 300, 256, 33, "f32"), "fused_kernel"),
+    (Workload("sh_sweep_bf16", 2, 4, 256, 512, 0, "bf16"), "sweep_kernel"),
+    (Workload("sh_sweep_local_f32", 1, 3, 300, 256, 33, "f32"), "sweep_kernel"),
 ]
+PATHS = {"fused_kernel": gspn.PATH_FUSED, "sweep_kernel": gspn.PATH_SWEEP}
 
 
 @pytest.mark.parametrize("wl,kernel", CASES, ids=[c[0].name for c in CASES])
 def test_shared_logits_match_oracle(wl, kernel, cuda_device):
+    gspn.debug_select_path(PATHS.get(kernel, gspn.PATH_AUTO))
+    try:
+        _check_shared(wl, kernel, cuda_device)
+    finally:
+        gspn.debug_select_path(gspn.PATH_AUTO)
+
+
+def _check_shared(wl, kernel, cuda_device):
     inp = inputs.make_inputs(wl, 77)
     # one logit plane set per batch entry: take channel 0 of the drawn logits
     zs = [t[:, :1].contiguous() for t in inp["wlogit"]]
