@@ -99,6 +99,21 @@ def test_large_planes_multi_cta_teams(H, W, g, dtype, cuda_device, fused_path):
     assert gspn.last_kernel_name() == ("fused_kernel" if (W * es) % 32 == 0 else "chain_kernel")
 
 
+@pytest.mark.parametrize("H,W", [(300, 256), (256, 512)])
+@pytest.mark.parametrize("d", [0, 1, 2, 3])
+def test_fused_single_direction(H, W, d, cuda_device, fused_path):
+    """One direction at a time on the fused kernel (its work queue then holds
+    one chain per plane)."""
+    wl = Workload("fdir", 1, 2, H, W, 0, "f32")
+    inp = inputs.make_inputs(wl, seed=10 + d)
+    dev = to_dev(inp, cuda_device)
+    y = gspn.forward_dir(dev["x"], dev["wlogit"][d], dev["lam"][d], dev["u"][d], d)
+    torch.cuda.synchronize()
+    assert gspn.last_kernel_name() == "fused_kernel"
+    ref = inp["u"][d].double().numpy() * oracle.hidden(inp["x"], inp["wlogit"][d], inp["lam"][d], d)
+    assert rel_err(y, ref) <= TOL["f32"]
+
+
 @pytest.mark.parametrize("path,kernel", [(1, "fused_kernel"), (2, "sweep_kernel")])
 def test_forced_timeout_is_reported_and_recovers(path, kernel, cuda_device):
     """A slot hand-over that never comes makes the kernel give up after its
