@@ -64,6 +64,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
+                    help="backward: time gspn_backward (gradients of sum(gy * y)) instead")
     ap.add_argument("--path", choices=["auto", "fused", "sweep"], default="auto",
                     help="large-plane kernel (auto: the fused kernel)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -367,6 +369,76 @@ def run_ours(args, wl):
     dist_close(world)
 
 
+# Backward pass: inputs x, 12 logits, 4 lambda, 4 u and gy are read; dx, 12
+# logit gradients, 4 lambda gradients and 4 u gradients are written.
+BACKWARD_ELEMS = 22 + 21
+
+
+def run_backward(args, wl):
+    """Times gspn_backward on the same synthetic workload: one step is the
+    whole backward call (its three kernels); the roofline is the call's
+    algorithmic bytes over its time, with the reverse-scan kernel's own time
+    beside it."""
+    rank, local, world = dist_init("nccl")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    gspn.load_library()
+    inp = make_inputs(wl, seed=rank, device=str(device), gen_device=str(device))
+    g = torch.Generator(device=str(device)).manual_seed(1000 + rank)
+    gy = torch.randn(inp["x"].shape, generator=g, device=device,
+                     dtype=torch.float32).to(inp["x"].dtype)
+    step = lambda: gspn.backward(inp["x"], inp["wlogit"], inp["lam"], inp["u"], gy,
+                                 wl.group_len)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = gspn.last_launch_count()
+    K = args.steps
+    kb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    for ev in kb + ke:
+        ev.record()
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.25)
+    t_start.record()
+    for i in range(K):
+        gspn.set_timing_events(kb[i], ke[i])
+        step()
+    t_end.record()
+    gspn.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = max_over_ranks(t_start.elapsed_time(t_end) / K, world, device)
+    scan_ms = max_over_ranks(statistics.mean(kb[i].elapsed_time(ke[i]) for i in range(K)),
+                             world, device)
+    peak, peak_kind = measured_hbm_peak()
+    alg_bytes = BACKWARD_ELEMS * wl.pixch * wl.esize
+    achieved = alg_bytes / (ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": "GSPN 4-dir backward (dx, dwlogit, dlam, du) Gpix·ch/s",
+            "pass": "backward", "value": wl.pixch * world / (ms * 1e-3) / 1e9, "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config_dict(wl, world),
+            "roofline": {"bound": "hbm", "kernel": "hidden_kernel+backward_kernel+round_kernel",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": achieved / peak,
+                         "algorithmic_bytes_per_launch": alg_bytes,
+                         "kernel_ms": ms, "backward_kernel_ms": scan_ms, "traffic": None},
+            "gpu_launches": launches_per_step * K,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    dist_close(world)
+
+
 def measure_e2e(args, wl, inp, device, world):
     """Same metric through gspn_forward_host: pinned host inputs copied in,
     y copied back, every step inside the timed region."""
@@ -406,6 +478,8 @@ def main():
         wl = wl.with_(C=args.C)
     if args.impl == "reference":
         run_reference(args, wl)
+    elif args.pass_ == "backward":
+        run_backward(args, wl)
     else:
         run_ours(args, wl)
 
