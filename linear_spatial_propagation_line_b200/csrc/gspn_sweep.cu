@@ -730,14 +730,18 @@ __device__ __forceinline__ void consume(const SweepParams& p, const View& sm, Ph
                     acc[j][kc >> 1] = (kc & 1) ? ptx::pk(x0, uh[j]) : ptx::pk(uh[j], x1);
                 }
                 if constexpr ((w & 3) == 3) {
-                    const int c0 = FWD ? s - 3 : L - 1 - s;
+                    // The last stage may run past the line (W a multiple of 4,
+                    // not of the stage): such groups of 4 steps are not added.
+                    const bool in = s < L;
+                    const int c0 = in ? (FWD ? s - 3 : L - 1 - s) : 0;
 #pragma unroll
                     for (int j = 0; j < kP; ++j) {
                         float x0, x1, x2, x3;
                         ptx::upk(acc[j][0], x0, x1);
                         ptx::upk(acc[j][1], x2, x3);
-                        ptx::red_add_v4_f32_if(own[j], slot + (size_t)(own[j] ? a[j] : 0) * W + c0,
-                                               x0, x1, x2, x3, pol_acc);
+                        ptx::red_add_v4_f32_if(own[j] && in,
+                                               slot + (size_t)(own[j] ? a[j] : 0) * W + c0, x0, x1,
+                                               x2, x3, pol_acc);
                     }
                 }
             }
@@ -1100,7 +1104,9 @@ size_t sweep_ctrl_bytes(int64_t planes) {
 bool sweep_plan(const Problem& pb, SweepPlan* sp) {
     const int es = pb.dtype == 0 ? 4 : 2;
     if (pb.H > 0x7fffffff / pb.W) return false;
-    if ((pb.W * es) % 16 != 0) return false;  // whole 16-byte horizontal stages, TMA strides
+    // 16-byte rows (TMA strides, whole 4-step output groups); a horizontal
+    // stage (32 bytes of columns) may run past W on zero-filled columns
+    if ((pb.W * es) % 16 != 0) return false;
     if (pb.planes() * 3 > 0x7fffffffLL) return false;
     if (pb.H < 2 * kP || pb.W < 2 * kP) return false;
     const int H = (int)pb.H, W = (int)pb.W;
@@ -1113,7 +1119,8 @@ bool sweep_plan(const Problem& pb, SweepPlan* sp) {
 
     const size_t slot_bytes = sizeof(float) * (size_t)H * W;
     const size_t l2_budget = (size_t)96 << 20;
-    for (int kc_max : {kMaxOwned}) {
+    {
+        const int kc_max = kMaxOwned;
         SweepPlan plan;
         memset(&plan, 0, sizeof(plan));
         int So[2];
@@ -1123,7 +1130,7 @@ bool sweep_plan(const Problem& pb, SweepPlan* sp) {
             while (So[o] <= 8 && round_up(ceil_div(K[o], So[o]), 8) > kc_max) So[o] *= 2;
             if (So[o] > 8) ok = false;
         }
-        if (!ok) continue;
+        if (!ok) return false;
         int S = 1;
         for (int o = 0; o < 2; ++o)
             if (nd[o] > 0 && So[o] > S) S = So[o];
@@ -1143,7 +1150,7 @@ bool sweep_plan(const Problem& pb, SweepPlan* sp) {
             if (sp_o > span) span = sp_o;
         }
         const int nw = ceil_div(span - 2 * kP, kStride);
-        if (!ok || nw > kMaxWarps) continue;
+        if (!ok || nw > kMaxWarps) return false;
         plan.nw = nw;
         plan.threads = 32 * (nw + 1);
         // A stage holds the exact span (rounded to 32 positions, so that every
@@ -1166,7 +1173,7 @@ bool sweep_plan(const Problem& pb, SweepPlan* sp) {
                 break;
             }
         }
-        if (plan.stages == 0) continue;
+        if (plan.stages == 0) return false;
         // work items of one plane
         int ipp = 0;
         for (int o = 0; o < 2; ++o) {
@@ -1180,7 +1187,7 @@ bool sweep_plan(const Problem& pb, SweepPlan* sp) {
         plan.ipp = ipp;
         int teams = pb.dtype == 0 ? max_teams<float, true>(plan)
                                   : max_teams<__nv_bfloat16, false>(plan);
-        if (teams <= 0) continue;
+        if (teams <= 0) return false;
         const int64_t items = pb.planes() * ipp;
         if (teams > items) teams = (int)items;
         const int64_t want_slots = (teams + ipp - 1) / ipp + 2;
