@@ -64,6 +64,9 @@ def _load():
             lib.gspn_oracle_hidden.argtypes = [_dp, _dp, _dp, i64, i64, i64, i64, i64,
                                                ctypes.c_int, ctypes.c_int, _dp]
             lib.gspn_oracle_hidden.restype = ctypes.c_int
+            lib.gspn_oracle_hidden_band.argtypes = [_dp, _dp, _dp, i64, i64, i64, i64, i64, i64,
+                                                    ctypes.c_int, ctypes.c_int, _dp]
+            lib.gspn_oracle_hidden_band.restype = ctypes.c_int
             lib.gspn_oracle_weights.argtypes = [_dp, i64, i64, i64, i64, ctypes.c_int, _dp]
             lib.gspn_oracle_weights.restype = ctypes.c_int
             arr4 = _dp * 4
@@ -105,6 +108,25 @@ def hidden(x, wlogit_d, lam_d, d: int, group_len: int = 0, nthreads: int = 0) ->
     h = np.empty_like(x)
     rc = _load().gspn_oracle_hidden(_ptr(x), _ptr(z), _ptr(lam), B, C, H, W, int(group_len),
                                     int(d), int(nthreads), _ptr(h))
+    if rc != 0:
+        raise ValueError(f"oracle rejected arguments (rc={rc})")
+    return h
+
+
+def hidden_band(x, wlogit_d, lam_d, d: int, radius: int, group_len: int = 0,
+                nthreads: int = 0) -> np.ndarray:
+    """h_d with a (2 radius + 1)-neighbour band instead of three neighbours;
+    wlogit_d: [B,C,2 radius + 1,H,W] (slot s = orthogonal offset s - radius).
+    radius = 1 is hidden(); radius >= K - 1 links every pixel to the whole
+    previous line."""
+    x = as_f64(x)
+    z = as_f64(wlogit_d)
+    lam = as_f64(lam_d)
+    B, C, H, W = x.shape
+    assert z.shape == (B, C, 2 * radius + 1, H, W) and lam.shape == x.shape
+    h = np.empty_like(x)
+    rc = _load().gspn_oracle_hidden_band(_ptr(x), _ptr(z), _ptr(lam), B, C, H, W, int(radius),
+                                         int(group_len), int(d), int(nthreads), _ptr(h))
     if rc != 0:
         raise ValueError(f"oracle rejected arguments (rc={rc})")
     return h

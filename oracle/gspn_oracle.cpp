@@ -177,6 +177,47 @@ void plane_backward(const Dir& dir, const double* x, const double* z3, const dou
     }
 }
 
+// ---- wider neighbourhoods ---------------------------------------------------
+// Section "如何设计一个高效的传播层" first states a direct method -- every pixel
+// links to all n pixels of the previous line, with weights normalised to sum
+// to 1 -- and sets it aside for its feature cost in favour of the three
+// neighbours above.  The banded form links pixel k to the previous line's
+// pixels k + o for |o| <= r: r = 1 is the tridiagonal layer, r >= K - 1 links
+// every pixel to the whole previous line (the direct method, a dense
+// row-stochastic w_i).  Logit slot s = 0 .. 2r is orthogonal offset s - r;
+// neighbours outside the line are dropped from the normaliser, as in section
+// "行随机矩阵".  Layout of the logits: [B][C][2r + 1][H][W].
+void plane_hidden_band(const Dir& dir, const double* x, const double* zb, const double* lam,
+                       int64_t g, int64_t r, double* h) {
+    const int64_t L = dir.L(), K = dir.K(), HW = dir.H * dir.W;
+    const int64_t nslot = 2 * r + 1;
+    std::vector<double> before(K), now(K), sig(nslot);
+    for (int64_t i = 0; i < L; ++i) {
+        const bool restart = group_start(dir, i, g);
+        for (int64_t k = 0; k < K; ++k) {
+            const int64_t p = dir.pixel(i, k);
+            double v = lam[p] * x[p];
+            if (!restart) {
+                double norm = 0.0;
+                for (int64_t s = 0; s < nslot; ++s) {
+                    const int64_t src = k + (s - r);
+                    sig[s] = (src >= 0 && src < K) ? logistic(zb[s * HW + p]) : 0.0;
+                    norm += sig[s];
+                }
+                double mix = 0.0;
+                for (int64_t s = 0; s < nslot; ++s) {
+                    const int64_t src = k + (s - r);
+                    if (src >= 0 && src < K) mix += (sig[s] / norm) * before[src];
+                }
+                v += mix;
+            }
+            now[k] = v;
+            h[p] = v;
+        }
+        before.swap(now);
+    }
+}
+
 template <class F>
 void parallel_planes(int64_t planes, int nthreads, F&& body) {
     if (nthreads <= 0) nthreads = (int)std::thread::hardware_concurrency();
@@ -216,6 +257,25 @@ int gspn_oracle_hidden(const double* x, const double* wlogit, const double* lam,
     const Dir dir{d, H, W};
     parallel_planes(B * C, nthreads, [&](int64_t q) {
         plane_hidden(dir, x + q * HW, wlogit + q * 3 * HW, lam + q * HW, group_len, h + q * HW);
+    });
+    return 0;
+}
+
+// Hidden state of one direction with a (2 * radius + 1)-neighbour band:
+// wlogit[B][C][2 * radius + 1][H][W], h[B][C][H][W].  radius = 1 is
+// gspn_oracle_hidden.  Returns 0, or -1 on a bad argument.
+int gspn_oracle_hidden_band(const double* x, const double* wlogit, const double* lam, int64_t B,
+                            int64_t C, int64_t H, int64_t W, int64_t radius, int64_t group_len,
+                            int d, int nthreads, double* h) {
+    if (!x || !wlogit || !lam || !h || bad_shape(B, C, H, W) || d < 0 || d > 3 ||
+        group_len < 0 || radius < 0)
+        return -1;
+    const int64_t HW = H * W;
+    const int64_t nslot = 2 * radius + 1;
+    const Dir dir{d, H, W};
+    parallel_planes(B * C, nthreads, [&](int64_t q) {
+        plane_hidden_band(dir, x + q * HW, wlogit + q * nslot * HW, lam + q * HW, group_len,
+                          radius, h + q * HW);
     });
     return 0;
 }

@@ -2,7 +2,8 @@
 
 Each case plants one mistake in a temporary copy of ``oracle/gspn_oracle.cpp``
 (on the CPU; nothing here touches a GPU), builds the copy, and runs the pin
-suite ``tests/test_oracle_pins.py`` against it in a subprocess.  The pins must
+suites (``tests/test_oracle_pins.py``, ``tests/test_oracle_backward_pins.py``
+and ``tests/test_oracle_band_pins.py``) against it in a subprocess.  The pins must
 fail for every mistake.  A case whose original text is no longer in the
 source fails too, so the list follows the oracle as it changes.
 """
@@ -43,6 +44,18 @@ MUTATIONS = [
      "carry[kn] += w[slot] * a[k];", "carry[k] += w[slot] * a[k];"),
     ("gate gradient uses the current line",
      "dw[slot] = a[k] * h[dir.pixel(i - 1, kn)];", "dw[slot] = a[k] * h[dir.pixel(i, kn)];"),
+    # wider neighbourhoods
+    ("band: neighbours outside the line kept in the normaliser",
+     "sig[s] = (src >= 0 && src < K) ? logistic(zb[s * HW + p]) : 0.0;",
+     "sig[s] = logistic(zb[s * HW + p]);"),
+    ("band: offsets mirrored",
+     "const int64_t src = k + (s - r);", "const int64_t src = k - (s - r);"),
+    ("band: in-place update reads the new line",
+     "if (src >= 0 && src < K) mix += (sig[s] / norm) * before[src];",
+     "if (src >= 0 && src < K) mix += (sig[s] / norm) * (src < k ? now[src] : before[src]);"),
+    ("band: last offset dropped",
+     "const int64_t nslot = 2 * r + 1;\n    std::vector<double> before",
+     "const int64_t nslot = 2 * r;\n    std::vector<double> before"),
 ]
 
 
@@ -55,7 +68,8 @@ def _run_pins_on_copy(tmp_path, src):
     (tmp_path / "oracle" / "gspn_oracle.cpp").write_text(src)
     env = dict(os.environ, PYTHONPATH=str(tmp_path))
     return subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                           "tests/test_oracle_pins.py", "tests/test_oracle_backward_pins.py"],
+                           "tests/test_oracle_pins.py", "tests/test_oracle_backward_pins.py",
+                           "tests/test_oracle_band_pins.py"],
                           cwd=tmp_path, env=env, capture_output=True, text=True, timeout=600)
 
 
